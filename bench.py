@@ -1,0 +1,476 @@
+"""Benchmark of one decode step of the paged-KV hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole hot path over one batch: the copy-on-write
+block copies (when the workload has shared blocks), the write of each
+sequence's new token into its slot, and paged decode attention (partition and
+reduce kernels).  The default workload is the Llama-3-8B-shaped GQA decode
+(256 sequences, 32 query / 8 KV heads, head dim 128, bf16, log-normal context
+lengths with median 1024 clipped to [128, 4096]).
+
+The metric is KV-read GB/s: the algorithmic K+V bytes a decode call reads
+(sum_b L_b * Hkv * 2 * D * element bytes) per step, divided by the step time,
+summed over ranks.  Rank 0 prints one JSON line.  ``--impl reference`` times the
+fp64 CPU oracle on the host cores instead (bounded sample of the same
+workload) and prints the same kind of line.
+
+Multi-GPU (torchrun): every rank decodes its own batch of the same shape
+(seed offset by rank); there is no exchange on the data path; the step time is
+the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from paged_kv_cache_464_b200 import inputs  # noqa: E402
+
+METRIC = "paged decode attention: KV-read GB/s (% of B200 HBM peak), seqs/s"
+DEFAULT_WORKLOAD = "llama3_8b_gqa"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def rank_seed(cfg: inputs.DecodeConfig, rank: int) -> int:
+    """Each rank draws its own batch of the workload's shape."""
+    return cfg.seed + 7919 * rank
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if any."""
+    path = os.path.join(ROOT, "profiles", f"pa_decode_{workload}.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms in a background process."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []   # (t, sm_mhz, max_mhz, reasons)
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            reasons = [n for n, v in zip(names, parts[5:9]) if v.lower() == "active"]
+            self.samples.append((time.time(), sm, mx, reasons))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        window = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not window:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({r for s in window for r in s[3]})
+        return {"sm_mhz": statistics.median(s[1] for s in window), "sm_max_mhz": max(s[2] for s in window),
+                "reasons": reasons, "samples": len(window)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def all_reduce_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def all_reduce_sum(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ our arm
+class Step:
+    """The device buffers of one workload and the step's calls through the C ABI."""
+
+    def __init__(self, case: inputs.DecodeCase, device):
+        from paged_kv_cache_464_b200 import capi
+        self.pa = capi
+        self.case = case
+        c = case.cfg
+        self.q = case.q.to(device)
+        self.k = case.k_cache.to(device)
+        self.v = case.v_cache.to(device)
+        self.key = case.key.to(device)
+        self.value = case.value.to(device)
+        self.slots = case.slot_mapping.to(device)
+        self.pairs = case.block_mapping.to(device)
+        self.bt = case.block_tables.to(device)
+        self.cl = case.context_lens.to(device)
+        self.out = torch.empty_like(self.q)
+        self.maxL = case.max_context_len
+        self.P = c.partition_size
+        ws = capi.decode_workspace_bytes(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, self.maxL, self.P)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+        self.has_pairs = case.block_mapping.numel() > 0
+        self.launches_per_step = self._count_launches()
+
+    def _count_launches(self):
+        c = self.case.cfg
+        P = self.pa.decode_partition_size(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, self.maxL, self.P)
+        split = math.ceil(self.maxL / P) > 1
+        return (1 if self.has_pairs else 0) + 1 + 1 + (1 if split else 0)
+
+    def pre(self):
+        if self.has_pairs:
+            self.pa.copy_blocks(self.k, self.v, self.pairs)
+        self.pa.reshape_and_cache(self.key, self.value, self.k, self.v, self.slots)
+
+    def decode(self):
+        self.pa.decode(self.q, self.k, self.v, self.bt, self.cl, self.case.scale, out=self.out,
+                       max_context_len=self.maxL, partition_size=self.P, workspace=self.ws)
+
+    def __call__(self):
+        self.pre()
+        self.decode()
+
+
+def run_ours(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = inputs.CONFIGS[args.workload]
+    case = inputs.make_case(cfg, seed=rank_seed(cfg, rank), with_post=False)
+    step = Step(case, device)
+    kv_bytes = case.kv_bytes()
+    stream = torch.cuda.current_stream()
+
+    sampler = ClockSampler(local).start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps; decode launches bracketed by events for the roofline
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step.pre()
+        ev_dec[i][0].record(stream)
+        step.decode()
+        ev_dec[i][1].record(stream)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(world)
+    elapsed_ms = t_start.elapsed_time(t_stop)
+    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+
+    # keep the GPU under the same load long enough for the clock sampler
+    soak_until = wall0 + 1.5
+    while time.time() < soak_until:
+        for _ in range(50):
+            step()
+        torch.cuda.synchronize()
+    wall_soak = time.time()
+    sampler.stop()
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = run_e2e(case, step, args.steps, args.warmup, device)
+
+    max_ms = all_reduce_max(elapsed_ms, world, device)
+    total_bytes = all_reduce_sum(float(kv_bytes), world, device)
+    total_seqs = all_reduce_sum(float(cfg.num_seqs), world, device)
+    e2e_ms = all_reduce_max(e2e["ms"], world, device)
+
+    if rank != 0:
+        return None
+    ms_per_step = max_ms / args.steps
+    value = total_bytes * args.steps / (max_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    dec_avg = statistics.mean(dec_ms)
+    achieved = kv_bytes / (dec_avg * 1e-3) / 1e9
+    clocks = sampler.summary(wall0, wall_soak)
+    traffic = profiled_traffic(args.workload)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.dtype,
+        "data": "synthetic (seeded N(0,1) Q/K/V, shuffled block pool)",
+        "config": {
+            "workload": cfg.name,
+            "description": cfg.description,
+            "num_seqs_per_gpu": cfg.num_seqs,
+            "num_heads": cfg.num_heads,
+            "num_kv_heads": cfg.num_kv_heads,
+            "head_dim": cfg.head_dim,
+            "block_size": cfg.block_size,
+            "sum_context_len": int(case.context_lens.sum()),
+            "kv_bytes_per_step_per_gpu": kv_bytes,
+            "partition_size": step.pa.decode_partition_size(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads,
+                                                            cfg.head_dim, step.maxL, step.P),
+            "step": ("copy_blocks + " if step.has_pairs else "") + "reshape_and_cache + decode",
+            "l2": f"inputs larger than L2: {kv_bytes / 2**20:.0f} MiB of KV per step vs 126 MiB L2, no flush",
+            "parallelism": f"replicas x{world}, no data-path collective",
+        },
+        "seqs_per_s": round(total_seqs * args.steps / (max_ms * 1e-3), 1),
+        "pct_hbm_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {
+            "kernel": "pa_decode (partition + reduce launches)",
+            "bound": "hbm",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6.65 TB/s",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "decode_ms_mean": round(dec_avg, 5),
+            "decode_ms_median": round(statistics.median(dec_ms), 5),
+        },
+        "e2e": {"value": round(total_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
+    return line
+
+
+def run_e2e(case, step, steps, warmup, device):
+    """Per step: inputs host->device from pinned memory, the step through the
+    public API, the output device->host into pinned memory."""
+    pa = step.pa
+    host = {k: getattr(case, k).pin_memory() for k in ("q", "key", "value", "slot_mapping", "block_mapping",
+                                                         "block_tables", "context_lens")}
+    dev = {"q": step.q, "key": step.key, "value": step.value, "slot_mapping": step.slots,
+           "block_mapping": step.pairs, "block_tables": step.bt, "context_lens": step.cl}
+    out_host = torch.empty(case.q.shape, dtype=case.q.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for k, t in host.items() if k != "block_mapping" or step.has_pairs)
+    d2h = out_host.numel() * out_host.element_size()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for k, t in host.items():
+            if k == "block_mapping" and not step.has_pairs:
+                continue
+            dev[k].copy_(t, non_blocking=True)
+        step()
+        out_host.copy_(step.out, non_blocking=True)
+
+    for _ in range(max(1, warmup)):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return {"ms": a.elapsed_time(b), "h2d": h2d, "d2h": d2h}
+
+
+# ------------------------------------------------------------------ oracle timings
+def _sample_case(case: inputs.DecodeCase, n: int) -> inputs.DecodeCase:
+    """The first n sequences of a case (same cache; copy pairs kept only for them)."""
+    import dataclasses
+    if n >= case.cfg.num_seqs:
+        return case
+    keep_pairs = case.block_mapping
+    if keep_pairs.numel():
+        rows = case.block_tables[:n].to(torch.int64)
+        used = set(rows[rows >= 0].tolist())
+        mask = torch.tensor([int(d) in used for d in keep_pairs[:, 1]], dtype=torch.bool)
+        keep_pairs = keep_pairs[mask]
+    return dataclasses.replace(case, cfg=dataclasses.replace(case.cfg, num_seqs=n), q=case.q[:n],
+                               key=case.key[:n], value=case.value[:n], slot_mapping=case.slot_mapping[:n],
+                               block_mapping=keep_pairs, block_tables=case.block_tables[:n],
+                               context_lens=case.context_lens[:n])
+
+
+def cpu_baseline(case, budget_s: float = 20.0):
+    """The oracle, as it stands, on the host cores: one step on a bounded sample.
+    The caches are cloned once outside the timed region (the step is idempotent)."""
+    import oracle
+    o = oracle.get()
+    k, v = case.k_cache.clone(), case.v_cache.clone()
+    # calibrate on a few sequences, then size the sample to the budget
+    n0 = min(4, case.cfg.num_seqs)
+    t = time.perf_counter()
+    o.step_inplace(_sample_case(case, n0), k, v)
+    per_seq = (time.perf_counter() - t) / n0
+    n = max(1, min(case.cfg.num_seqs, int(budget_s / 2 / max(per_seq, 1e-6))))
+    sample = _sample_case(case, n)
+    best = None
+    reps = 0
+    t_all = time.perf_counter()
+    while reps < 3 and (reps == 0 or time.perf_counter() - t_all < budget_s / 2):
+        t = time.perf_counter()
+        o.step_inplace(sample, k, v)
+        dt = time.perf_counter() - t
+        best = dt if best is None else min(best, dt)
+        reps += 1
+    return {"value": round(sample.kv_bytes() / best / 1e9, 4), "unit": "GB/s", "cores": o.num_threads,
+            "kind": "oracle", "seqs_per_s": round(n / best, 3),
+            "sample": f"first {n} of {case.cfg.num_seqs} sequences of the same workload, one full step "
+                      f"(copies, new-token write, fp64 decode), best of {reps}"}
+
+
+def run_reference(args, world, rank):
+    """The fp64 oracle as the reference arm, on the host cores, rank 0 only."""
+    if rank != 0:
+        return None
+    import oracle
+    o = oracle.get()
+    cfg = inputs.CONFIGS[args.workload]
+    case = inputs.make_case(cfg, seed=rank_seed(cfg, 0), with_post=False)
+    k, v = case.k_cache.clone(), case.v_cache.clone()
+    # size each step so that warm-up + timed steps take about `ref_budget` seconds
+    n0 = min(4, cfg.num_seqs)
+    t = time.perf_counter()
+    o.step_inplace(_sample_case(case, n0), k, v)
+    per_seq = (time.perf_counter() - t) / n0
+    per_step_budget = args.ref_budget / max(1, args.steps + args.warmup)
+    n = max(1, min(cfg.num_seqs, int(per_step_budget / max(per_seq, 1e-6))))
+    sample = _sample_case(case, n)
+    for _ in range(args.warmup):
+        o.step_inplace(sample, k, v)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        o.step_inplace(sample, k, v)
+    el = time.perf_counter() - t0
+    value = sample.kv_bytes() * args.steps / el / 1e9
+    desc = (f"first {n} of {cfg.num_seqs} sequences per step (copies, new-token write, fp64 decode), "
+            f"{o.num_threads} threads")
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "description": cfg.description, "sample_seqs_per_step": n},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": o.num_threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(inputs.CONFIGS))
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds for the CPU-baseline sample")
+    ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds for the whole reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+        else:
+            line = run_ours(args, world, rank, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

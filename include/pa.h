@@ -1,0 +1,186 @@
+/*
+ * pa.h -- C ABI of libpa_b200.so: paged-KV decode attention on NVIDIA B200
+ * (sm_100a).
+ *
+ * The library implements the decode-time hot path of a paged KV cache as
+ * described by these web pages (cited by title and section):
+ *   [A] "vLLM推理引擎深度解析：从PagedAttention原理到高吞吐量部署的工程实践"
+ *       §三 PagedAttention：虚拟内存思想应用于KV Cache (block pool, per-request
+ *       block table, append_token, share_prefix with reference counts);
+ *       §五 优化的注意力计算 (PagedAttention.forward: gather K/V through the
+ *       block table, scores, 1/sqrt(head_dim) scale, softmax, weighted V; the
+ *       new token's K/V is written into the cache).
+ *   [B] "vLLM 原理与源码阅读": PagedAttention 核心思想 (logical -> physical
+ *       block map); Block 管理器 (block table per request, block size 16 by
+ *       default, copy-on-write of a shared block).
+ *   [C] "vLLM推理引擎深度实战：…" §1.2 PagedAttention原理 (block table, allocation
+ *       failure reported as an error).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer argument except `stream` and the `detail` out-parameter of
+ *   pa_get_device_error is DEVICE memory owned by the caller.  The library
+ *   allocates no device or host memory and keeps no state across calls except
+ *   one device error word per GPU (see pa_get_device_error).
+ * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *   NULL = the legacy default stream).  The returned status covers host-side
+ *   argument checks and the launch itself (cudaGetLastError).  Problems that
+ *   only the GPU can see (a block id or slot out of range, a context length
+ *   beyond the table) never fault or trap: the kernel skips the bad access and
+ *   records the first such problem in the device error word.
+ * - KV cache layout: two separate tensors k_cache and v_cache, each
+ *   [num_blocks][block_size][num_kv_heads][head_dim], row-major, contiguous
+ *   (token-major inside a block, the per-block layout of [A] §五 with the K/V
+ *   axis split into two tensors).  block_size must be 16.  One (token, KV head)
+ *   row must be 256 bytes: head_dim 64 for PA_F32, 128 for PA_F16 / PA_BF16.
+ *   Cache base addresses must be 16-byte aligned.
+ * - A slot is a flat token index into the pool: slot = physical_block *
+ *   block_size + offset ([A] §三 append_token: a new token goes to the next
+ *   free offset of the sequence's last block, else to a newly allocated block).
+ */
+#ifndef PA_B200_PA_H
+#define PA_B200_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype_t;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_NULL = 1,       /* a required pointer is NULL */
+  PA_ERR_DTYPE = 2,      /* unknown dtype */
+  PA_ERR_SHAPE = 3,      /* unsupported or inconsistent sizes (see each call) */
+  PA_ERR_WORKSPACE = 4,  /* split-K workspace missing or too small */
+  PA_ERR_CUDA = 5,       /* a CUDA runtime/driver call or the launch failed */
+  PA_ERR_ALIGN = 6,      /* a pointer is not aligned as required */
+} pa_status_t;
+
+/* Kinds recorded in the device error word (pa_get_device_error). */
+typedef enum {
+  PA_DEV_OK = 0,
+  PA_DEV_BAD_BLOCK_ID = 1,     /* block id outside [0, num_blocks); detail = the id */
+  PA_DEV_BAD_SLOT = 2,         /* slot >= num_blocks * block_size; detail = the slot */
+  PA_DEV_COPY_CONFLICT = 3,    /* copy pair skipped (dst repeated or read by a pair); detail = pair index */
+  PA_DEV_BAD_CONTEXT_LEN = 4,  /* context_len < 0, > max_context_len or > table capacity; detail = seq */
+  PA_DEV_WAIT_TIMEOUT = 5,     /* an internal bounded wait gave up; detail = CTA index */
+} pa_device_error_t;
+
+/*
+ * pa_reshape_and_cache -- write each new token's K and V rows into its slot.
+ * ([A] §五: the current token's k/v join the cache; [A] §三 append_token.)
+ *
+ * key, value    [num_tokens][num_kv_heads][head_dim], contiguous, cache dtype.
+ * k_cache, v_cache  the caches (layout above); modified in place.
+ * slot_mapping  [num_tokens] int64: destination slot of token i.  slot < 0
+ *               means "no write" (padding).  slot >= num_blocks*block_size is
+ *               skipped and recorded as PA_DEV_BAD_SLOT.  Slots must be
+ *               distinct; with duplicates the written row is unspecified.
+ * The copy is bit-exact: every byte of each row is moved unchanged, and no
+ * other cache byte is touched.
+ * Errors: PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE (num_tokens < 0, block_size
+ * != 16, row not 256 bytes, num_blocks <= 0), PA_ERR_ALIGN (16-byte
+ * alignment of key/value/caches), PA_ERR_CUDA.  num_tokens == 0 is a no-op.
+ */
+pa_status_t pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                                 const int64_t *slot_mapping, int num_tokens, int64_t num_blocks,
+                                 int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype,
+                                 void *stream);
+
+/*
+ * pa_decode_partition_size -- the partition size (tokens per split-K piece)
+ * that pa_decode will use for these arguments.  `requested` > 0 is returned
+ * unchanged (it must be a positive multiple of block_size); 0 selects the
+ * library's choice.  Returns -1 for invalid arguments.
+ */
+int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                             int max_context_len, int requested);
+
+/*
+ * pa_decode_workspace_bytes -- bytes of split-K workspace pa_decode needs
+ * (0 when no sequence can span more than one partition).  Same arguments as
+ * pa_decode_partition_size.  Returns 0 for invalid arguments as well; callers
+ * that care check pa_decode_partition_size first.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int max_context_len, int requested_partition_size);
+
+/*
+ * pa_decode -- single-query attention for every sequence over its paged KV
+ * cache ([A] §五 PagedAttention.forward; [B] PagedAttention 核心思想).
+ *
+ * For sequence b, query head h, KV head g = h / (num_heads / num_kv_heads):
+ *   K_t, V_t  = row (physical block block_tables[b][t / 16], offset t % 16,
+ *               head g) of k_cache / v_cache, for t < context_lens[b]
+ *   out[b][h] = sum_t softmax_t(scale * <q[b][h], K_t>) * V_t
+ * Accumulation is fp32; the output is rounded to the cache dtype (nearest
+ * even).  context_lens[b] == 0 gives an all-zero row.
+ *
+ * out           [num_seqs][num_heads][head_dim], cache dtype (written).
+ * q             [num_seqs][num_heads][head_dim], cache dtype.
+ * block_tables  [num_seqs][max_blocks_per_seq] int32; entries at or past
+ *               ceil(context_lens[b] / 16) are never read.
+ * context_lens  [num_seqs] int32; each must be <= max_context_len and
+ *               <= max_blocks_per_seq * 16 (else PA_DEV_BAD_CONTEXT_LEN and
+ *               that row is not written).
+ * max_context_len  host-side upper bound of context_lens (sizes the grid).
+ * scale         softmax scale (1/sqrt(head_dim) in the pages).
+ * partition_size   0 = library's choice, else a positive multiple of 16:
+ *               sequences longer than it are split into pieces that are
+ *               combined by a second (reduce) kernel through `workspace`.
+ * workspace     device buffer of >= pa_decode_workspace_bytes(...) bytes,
+ *               256-byte aligned (may be NULL when that is 0).  Its contents
+ *               need no initialisation and are scratch after the call.
+ * Errors: PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE (num_heads % num_kv_heads,
+ * group size not in {1,2,4,8}, row not 256 bytes, block_size != 16, bad
+ * partition_size, negative sizes), PA_ERR_WORKSPACE, PA_ERR_ALIGN (16-byte
+ * alignment of q/out/caches, 256 of workspace), PA_ERR_CUDA.
+ */
+pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *context_lens, int num_seqs, int num_heads,
+                      int max_context_len, float scale, int partition_size, void *workspace,
+                      size_t workspace_bytes, int64_t num_blocks, int block_size, int num_kv_heads,
+                      int head_dim, pa_dtype_t dtype, void *stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copies ([B] Block 管理器, item 3:
+ * when a request writes to a block that several requests share, the block is
+ * copied first and the request's table is pointed at the copy; the caller
+ * keeps the reference counts and rewrites the tables).
+ *
+ * block_mapping [num_pairs][2] int64 (src, dst): block src of both caches is
+ * copied whole (block_size * num_kv_heads * head_dim elements, bit-exact) to
+ * block dst.  A pair is skipped and recorded as PA_DEV_BAD_BLOCK_ID if an id
+ * is outside [0, num_blocks), or as PA_DEV_COPY_CONFLICT if its dst is the dst
+ * of another pair or the src of any pair (itself included); all other pairs
+ * are carried out, independently of their order.  The conflict check reads
+ * all pairs from every CTA: cost O(num_pairs^2) reads of 16 bytes.
+ * Errors: PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_CUDA.
+ * num_pairs == 0 is a no-op.
+ */
+pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
+                           int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                           pa_dtype_t dtype, void *stream);
+
+/*
+ * pa_get_device_error -- synchronise `stream`, then return the first problem a
+ * kernel recorded on the current device since the last clear (a
+ * pa_device_error_t; 0 = none).  `detail` (host pointer, may be NULL)
+ * receives the offending value.  clear != 0 resets the word to 0.
+ * Returns -1 if a CUDA call fails.
+ */
+int pa_get_device_error(void *stream, int64_t *detail, int clear);
+
+/* pa_status_string -- a static, human-readable name of a status. */
+const char *pa_status_string(pa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_B200_PA_H */

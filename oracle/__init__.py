@@ -135,14 +135,17 @@ class Oracle:
         new token's write, then decode.  Returns (out, k_cache, v_cache)."""
         k = case.k_cache.clone()
         v = case.v_cache.clone()
+        return self.step_inplace(case, k, v), k, v
+
+    def step_inplace(self, case, k, v):
+        """The same step on caches the caller owns (modified in place); returns out."""
         rc = self.copy_blocks(k, v, case.block_mapping)
         if rc:
             raise OracleError(rc)
         rc = self.reshape_and_cache(k, v, case.key, case.value, case.slot_mapping)
         if rc:
             raise OracleError(rc)
-        out = self.paged_decode(case.q, k, v, case.block_tables, case.context_lens, case.scale)
-        return out, k, v
+        return self.paged_decode(case.q, k, v, case.block_tables, case.context_lens, case.scale)
 
     @property
     def num_threads(self) -> int:

@@ -1,0 +1,295 @@
+// pa.cu -- the C ABI of libpa_b200.so (declared in include/pa.h): host-side
+// argument checks, TMA descriptor encoding and kernel launches.  The kernels
+// themselves live in pa_cache_ops.cuh and pa_decode.cuh, compiled here as one
+// translation unit so that the per-device error word needs no separate
+// device linking.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "pa.h"
+#include "pa_cache_ops.cuh"
+#include "pa_decode.cuh"
+
+namespace {
+
+using pa::kBlockSize;
+using pa::kRowBytes;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int elem_bytes(pa_dtype_t dt) {
+  switch (dt) {
+    case PA_F32: return 4;
+    case PA_F16:
+    case PA_BF16: return 2;
+  }
+  return 0;
+}
+
+pa_status_t cache_shape_status(int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                               pa_dtype_t dtype) {
+  const int es = elem_bytes(dtype);
+  if (es == 0) return PA_ERR_DTYPE;
+  if (num_blocks <= 0 || num_blocks > INT32_MAX || block_size != kBlockSize || num_kv_heads <= 0 ||
+      head_dim * es != kRowBytes)
+    return PA_ERR_SHAPE;
+  return PA_OK;
+}
+
+pa_status_t launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// The cache [NB][16][Hkv][256 B] seen as a 5-D byte tensor
+// {128 B, 2 halves, Hkv, 16 tokens, NB}; the box is one (block, KV head) tile:
+// {128, 2, 1, 16, 1} = 4 KiB, landing 128-byte swizzled.
+bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int num_kv_heads) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[5] = {128, kRowBytes / 128, (cuuint64_t)num_kv_heads, (cuuint64_t)kBlockSize,
+                              (cuuint64_t)num_blocks};
+  const cuuint64_t strides[4] = {128, (cuuint64_t)kRowBytes, (cuuint64_t)num_kv_heads * kRowBytes,
+                                 (cuuint64_t)kBlockSize * num_kv_heads * kRowBytes};
+  const cuuint32_t box[5] = {128, kRowBytes / 128, 1, kBlockSize, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(cache), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- decode planning
+int resolve_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_context_len,
+                           int requested) {
+  (void)num_seqs;
+  (void)num_heads;
+  (void)num_kv_heads;
+  (void)head_dim;
+  if (max_context_len < 0 || requested < 0) return -1;
+  if (requested > 0) return requested % kBlockSize == 0 ? requested : -1;
+  if (max_context_len <= 512) return max_context_len <= kBlockSize ? kBlockSize
+                                                                    : (max_context_len + kBlockSize - 1) / kBlockSize * kBlockSize;
+  return 512;
+}
+
+int max_partitions(int max_context_len, int partition_size) {
+  const int np = (max_context_len + partition_size - 1) / partition_size;
+  return np < 1 ? 1 : np;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WorkspaceLayout {
+  size_t m_off, l_off, o_off, bytes;
+};
+
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int np) {
+  WorkspaceLayout w{};
+  if (np <= 1) return w;
+  const size_t rows = (size_t)num_seqs * num_heads * np;
+  w.m_off = 0;
+  w.l_off = align256(rows * sizeof(float));
+  w.o_off = w.l_off + align256(rows * sizeof(float));
+  w.bytes = w.o_off + align256(rows * head_dim * sizeof(float));
+  return w;
+}
+
+template <typename T, int G>
+pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
+                          cudaStream_t stream) {
+  using SM = pa::DecodeSmem<T, G>;
+  auto kernel = pa::pa_decode_partition_kernel<T, G>;
+  // the attribute is per device; setting it on every call costs ~a microsecond of host time
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
+    return PA_ERR_CUDA;
+  const long long grid = (long long)p.num_seqs * p.num_kv_heads * p.max_partitions;
+  if (grid == 0) return PA_OK;
+  if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  kernel<<<(unsigned)grid, pa::kDecodeThreads, SM::kAlloc, stream>>>(mk, mv, p);
+  pa_status_t st = launch_status();
+  if (st != PA_OK || p.max_partitions <= 1) return st;
+  const long long rows = (long long)p.num_seqs * p.num_heads;
+  pa::pa_decode_reduce_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
+  return launch_status();
+}
+
+template <typename T>
+pa_status_t dispatch_group(int group, const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
+                           cudaStream_t s) {
+  switch (group) {
+    case 1: return launch_decode<T, 1>(mk, mv, p, s);
+    case 2: return launch_decode<T, 2>(mk, mv, p, s);
+    case 4: return launch_decode<T, 4>(mk, mv, p, s);
+    case 8: return launch_decode<T, 8>(mk, mv, p, s);
+  }
+  return PA_ERR_SHAPE;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status_t pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                                 const int64_t *slot_mapping, int num_tokens, int64_t num_blocks,
+                                 int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype,
+                                 void *stream) {
+  pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_SHAPE;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_NULL;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_ALIGN;
+  const int chunks_per_slot = num_kv_heads * (kRowBytes / 16);
+  const long long total = (long long)num_tokens * chunks_per_slot;
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  pa::reshape_and_cache_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+      (const uint4 *)key, (const uint4 *)value, (uint4 *)k_cache, (uint4 *)v_cache, slot_mapping, num_tokens,
+      chunks_per_slot, (long long)num_blocks * block_size);
+  return launch_status();
+}
+
+int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_context_len,
+                             int requested) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return -1;
+  return resolve_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, requested);
+}
+
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_context_len,
+                                 int requested_partition_size) {
+  const int P = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                         requested_partition_size);
+  if (P <= 0) return 0;
+  return workspace_layout(num_seqs, num_heads, head_dim, max_partitions(max_context_len, P)).bytes;
+}
+
+pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                      int num_seqs, int num_heads, int max_context_len, float scale, int partition_size,
+                      void *workspace, size_t workspace_bytes, int64_t num_blocks, int block_size,
+                      int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream) {
+  pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 || max_blocks_per_seq < 0 ||
+      num_heads % num_kv_heads != 0 || !std::isfinite(scale))
+    return PA_ERR_SHAPE;
+  const int group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_SHAPE;
+  if ((long long)max_blocks_per_seq * kBlockSize > INT32_MAX) return PA_ERR_SHAPE;
+  const int P = resolve_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                       partition_size);
+  if (P <= 0) return PA_ERR_SHAPE;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !context_lens || (max_blocks_per_seq > 0 && !block_tables))
+    return PA_ERR_NULL;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PA_ERR_ALIGN;
+  const int np = max_partitions(max_context_len, P);
+  const WorkspaceLayout ws = workspace_layout(num_seqs, num_heads, head_dim, np);
+  if (ws.bytes > 0) {
+    if (!workspace || workspace_bytes < ws.bytes) return PA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return PA_ERR_ALIGN;
+  }
+
+  CUtensorMap mk, mv;
+  if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads) ||
+      !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads))
+    return PA_ERR_CUDA;
+
+  pa::DecodeParams p{};
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  char *w = static_cast<char *>(workspace);
+  p.ws_m = ws.bytes ? reinterpret_cast<float *>(w + ws.m_off) : nullptr;
+  p.ws_l = ws.bytes ? reinterpret_cast<float *>(w + ws.l_off) : nullptr;
+  p.ws_o = ws.bytes ? reinterpret_cast<float *>(w + ws.o_off) : nullptr;
+  p.num_blocks = num_blocks;
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context_len = max_context_len;
+  p.partition_size = P;
+  p.max_partitions = np;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (dtype) {
+    case PA_F32: return dispatch_group<float>(group, mk, mv, p, s);
+    case PA_F16: return dispatch_group<__half>(group, mk, mv, p, s);
+    case PA_BF16: return dispatch_group<__nv_bfloat16>(group, mk, mv, p, s);
+  }
+  return PA_ERR_DTYPE;
+}
+
+pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
+                           int64_t num_blocks, int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype,
+                           void *stream) {
+  pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0 || num_pairs > 65535 * 1024) return PA_ERR_SHAPE;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_mapping) return PA_ERR_NULL;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8)) return PA_ERR_ALIGN;
+  const int chunks_per_block = kBlockSize * num_kv_heads * (kRowBytes / 16);
+  pa::copy_blocks_kernel<<<dim3((unsigned)num_pairs, 2), 256, 0, (cudaStream_t)stream>>>(
+      (uint4 *)k_cache, (uint4 *)v_cache, (const long long *)block_mapping, num_pairs, (long long)num_blocks,
+      chunks_per_block);
+  return launch_status();
+}
+
+int pa_get_device_error(void *stream, int64_t *detail, int clear) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return -1;
+  int code = 0;
+  long long d = 0;
+  if (cudaMemcpyFromSymbol(&code, pa::g_error_code, sizeof(int)) != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(&d, pa::g_error_detail, sizeof(long long)) != cudaSuccess) return -1;
+  if (detail) *detail = d;
+  if (clear) {
+    const int zero = 0;
+    const long long zd = 0;
+    if (cudaMemcpyToSymbol(pa::g_error_code, &zero, sizeof(int)) != cudaSuccess) return -1;
+    if (cudaMemcpyToSymbol(pa::g_error_detail, &zd, sizeof(long long)) != cudaSuccess) return -1;
+  }
+  return code;
+}
+
+const char *pa_status_string(pa_status_t status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_NULL: return "PA_ERR_NULL: a required pointer is NULL";
+    case PA_ERR_DTYPE: return "PA_ERR_DTYPE: unknown dtype";
+    case PA_ERR_SHAPE: return "PA_ERR_SHAPE: unsupported or inconsistent sizes";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: split-K workspace missing or too small";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case PA_ERR_ALIGN: return "PA_ERR_ALIGN: a pointer is not aligned as required";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

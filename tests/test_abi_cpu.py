@@ -1,0 +1,114 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/pa.h declares, and host-side validation returns the documented codes
+before any CUDA call is made."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from paged_kv_cache_464_b200 import build
+    build.build()
+    from paged_kv_cache_464_b200 import capi
+    return capi
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("pa_reshape_and_cache", "pa_decode", "pa_copy_blocks"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(capi):
+    out = subprocess.run(["nm", "-D", "--defined-only", capi.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    assert sorted(capi.EXPORTED) == declared_functions()
+
+
+def test_header_compiles_as_c():
+    src = f'#include "{HEADER}"\nint main(void){{ return (int)PA_OK; }}\n'
+    r = subprocess.run(["gcc", "-x", "c", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-"], input=src,
+                       text=True, capture_output=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_status_strings(capi):
+    for code in range(7):
+        assert capi.raw.pa_status_string(code).decode().startswith("PA_")
+
+
+def test_partition_and_workspace_sizes(capi):
+    # explicit partition sizes must be multiples of the block size
+    assert capi.decode_partition_size(8, 64, 8, 128, 32768, 512) == 512
+    assert capi.decode_partition_size(8, 64, 8, 128, 32768, 500) == -1
+    assert capi.decode_partition_size(8, 64, 8, 128, -1, 0) == -1
+    # automatic choice: one partition when short, split when long
+    p = capi.decode_partition_size(4, 4, 4, 64, 100, 0)
+    assert p >= 100 and p % 16 == 0
+    assert capi.decode_workspace_bytes(4, 4, 4, 64, 100, 0) == 0
+    p = capi.decode_partition_size(8, 64, 8, 128, 32768, 0)
+    npart = -(-32768 // p)
+    ws = capi.decode_workspace_bytes(8, 64, 8, 128, 32768, 0)
+    assert ws >= 8 * 64 * npart * (128 + 2) * 4
+    # long-context workload at partition 512: 8*64*64 rows of (128 + 2) floats
+    assert capi.decode_workspace_bytes(8, 64, 8, 128, 32768, 512) >= 8 * 64 * 64 * 130 * 4
+
+
+def _decode(capi, **kw):
+    args = dict(out=16, q=16, k=16, v=16, bt=16, mbs=4, cl=16, S=2, Hq=4, maxL=64, scale=0.125, P=0,
+                ws=None, wsb=0, NB=8, bs=16, Hkv=4, D=64, dt=0)
+    args.update(kw)
+    a = args
+    return capi.raw.pa_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["mbs"], a["cl"], a["S"], a["Hq"],
+                              a["maxL"], a["scale"], a["P"], a["ws"], a["wsb"], a["NB"], a["bs"], a["Hkv"],
+                              a["D"], a["dt"], None)
+
+
+def test_decode_host_validation(capi):
+    PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE, PA_ERR_WORKSPACE, PA_ERR_ALIGN = 1, 2, 3, 4, 6
+    assert _decode(capi, dt=7) == PA_ERR_DTYPE
+    assert _decode(capi, bs=32) == PA_ERR_SHAPE                 # block size must be 16
+    assert _decode(capi, D=128) == PA_ERR_SHAPE                 # fp32 row must be 256 B
+    assert _decode(capi, dt=2, D=64) == PA_ERR_SHAPE            # bf16 needs D=128
+    assert _decode(capi, Hq=6) == PA_ERR_SHAPE                  # Hq % Hkv
+    assert _decode(capi, Hq=64) == PA_ERR_SHAPE                 # group 16 not built
+    assert _decode(capi, P=24) == PA_ERR_SHAPE                  # partition not a multiple of 16
+    assert _decode(capi, S=-1) == PA_ERR_SHAPE
+    assert _decode(capi, NB=0) == PA_ERR_SHAPE
+    assert _decode(capi, scale=float("nan")) == PA_ERR_SHAPE
+    assert _decode(capi, q=None) == PA_ERR_NULL
+    assert _decode(capi, out=8) == PA_ERR_ALIGN
+    assert _decode(capi, maxL=4096, P=512) == PA_ERR_WORKSPACE  # split needs a workspace
+    assert _decode(capi, maxL=4096, P=512, ws=256, wsb=10) == PA_ERR_WORKSPACE
+    assert _decode(capi, S=0) == 0                              # nothing to do
+
+
+def test_cache_ops_host_validation(capi):
+    r = capi.raw
+    # (key, value, k_cache, v_cache, slots, T, NB, bs, Hkv, D, dtype, stream)
+    assert r.pa_reshape_and_cache(16, 16, 16, 16, 16, 0, 8, 16, 4, 64, 0, None) == 0
+    assert r.pa_reshape_and_cache(16, 16, 16, 16, 16, -1, 8, 16, 4, 64, 0, None) == 3
+    assert r.pa_reshape_and_cache(None, 16, 16, 16, 16, 4, 8, 16, 4, 64, 0, None) == 1
+    assert r.pa_reshape_and_cache(16, 16, 24, 16, 16, 4, 8, 16, 4, 64, 0, None) == 6
+    assert r.pa_reshape_and_cache(16, 16, 16, 16, 16, 4, 8, 16, 4, 64, 3, None) == 2
+    # (k_cache, v_cache, mapping, P, NB, bs, Hkv, D, dtype, stream)
+    assert r.pa_copy_blocks(16, 16, 16, 0, 8, 16, 4, 64, 0, None) == 0
+    assert r.pa_copy_blocks(16, 16, None, 2, 8, 16, 4, 64, 0, None) == 1
+    assert r.pa_copy_blocks(16, 16, 16, -2, 8, 16, 4, 64, 0, None) == 3
+    assert r.pa_copy_blocks(16, 16, 16, 2, 8, 16, 4, 96, 1, None) == 3
