@@ -168,6 +168,47 @@ pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_ma
                            pa_dtype_t dtype, void *stream);
 
 /*
+ * PA_STATIC_WORKSPACE_BYTES -- size of the split-K scratch that the library
+ * itself owns for pa_decode_static_workspace: 64 MiB in every GPU that loads
+ * the library, held until the process exits.
+ */
+#define PA_STATIC_WORKSPACE_BYTES ((size_t)64 << 20)
+
+/*
+ * pa_decode_static_workspace -- pa_decode without a caller-provided workspace
+ * and without allocating anything.  The source pages have no counterpart to
+ * this call: it exists for users of this library who cannot allocate device
+ * memory at the point where they decode -- for example a plugin running inside
+ * a serving process whose own allocator owns all device memory and hands out
+ * no side buffers, or a latency-critical loop that must not call cudaMalloc or
+ * cudaFree because those calls can synchronise the device.
+ *
+ * Arguments, results and errors are those of pa_decode, minus workspace and
+ * workspace_bytes.  The split-K scratch is a library-owned device array of
+ * PA_STATIC_WORKSPACE_BYTES; a call whose pa_decode_workspace_bytes(...)
+ * exceeds it returns PA_ERR_WORKSPACE without launching anything (e.g. the
+ * 256-sequence, 32-head, 4096-token workload at partition 512 needs 33 MiB and
+ * fits; 4096 sequences of that shape would not).  The call allocates no device
+ * or host memory: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Set-up: the first accepted call on a device (that device current) looks up
+ * the array's device address with cudaGetSymbolAddress and caches it; make
+ * that first call before any stream capture.  Later calls do no set-up.
+ *
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents.  Nothing in it needs clearing between calls (each call
+ * writes every scratch entry it later reads), but calls whose kernels overlap
+ * on the GPU -- on different streams, or from different host threads -- race on
+ * the array and give wrong results.  Serialise them (one stream, or events).
+ */
+pa_status_t pa_decode_static_workspace(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                       const int32_t *block_tables, int max_blocks_per_seq,
+                                       const int32_t *context_lens, int num_seqs, int num_heads,
+                                       int max_context_len, float scale, int partition_size,
+                                       int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                                       pa_dtype_t dtype, void *stream);
+
+/*
  * pa_get_device_error -- synchronise `stream`, then return the first problem a
  * kernel recorded on the current device since the last clear (a
  * pa_device_error_t; 0 = none).  `detail` (host pointer, may be NULL)

@@ -28,6 +28,9 @@ _lib.pa_decode_workspace_bytes.restype = _SZ
 _lib.pa_decode_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.pa_decode.restype = _I
 _lib.pa_decode.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _P, _SZ, _I64, _I, _I, _I, _I, _P]
+_lib.pa_decode_static_workspace.restype = _I
+_lib.pa_decode_static_workspace.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _I64, _I, _I, _I, _I,
+                                            _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I64, _I, _I, _I, _I, _P]
 _lib.pa_get_device_error.restype = _I
@@ -36,7 +39,8 @@ _lib.pa_status_string.restype = ctypes.c_char_p
 _lib.pa_status_string.argtypes = [_I]
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
+            "pa_decode_static_workspace", "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
+STATIC_WORKSPACE_BYTES = 64 << 20   # PA_STATIC_WORKSPACE_BYTES in include/pa.h
 
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 DEVICE_ERRORS = {0: "ok", 1: "block id out of range", 2: "slot out of range", 3: "copy pair conflict",
@@ -140,6 +144,36 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
                           _dev(block_tables, "block_tables"), block_tables.shape[1],
                           _dev(context_lens, "context_lens"), S, hq, max_context_len, float(scale),
                           partition_size, ws_ptr, ws_bytes, nb, bs, hkv, d, dt, _stream(stream)), "pa_decode")
+    return out
+
+
+def decode_static_workspace(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                            block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                            out: Optional[torch.Tensor] = None, *, max_context_len: int,
+                            partition_size: int = 0, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """``decode`` for callers that cannot allocate device memory: the split-K
+    scratch is the library's own fixed array (STATIC_WORKSPACE_BYTES per GPU),
+    so the library allocates nothing.  ``out`` must be given by such callers
+    (it is allocated here only as a convenience when omitted).  Calls that
+    overlap on the GPU share the array and race; the first call on a device
+    looks up the array's address and should precede any stream capture."""
+    nb, bs, hkv, d, dt = _cache_args(k_cache, v_cache)
+    S, hq, dq = q.shape
+    if dq != d or q.dtype != k_cache.dtype:
+        raise ValueError("q must be [S, num_heads, head_dim] with the cache dtype")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("block_tables must be [S, max_blocks_per_seq] and context_lens [S]")
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    _check(_lib.pa_decode_static_workspace(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"), S, hq,
+        max_context_len, float(scale), partition_size, nb, bs, hkv, d, dt, _stream(stream)),
+        "pa_decode_static_workspace")
     return out
 
 

@@ -263,6 +263,52 @@ pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_ma
   return launch_status();
 }
 
+// ---------------------------------------------------------------- no-allocation decode
+// Split-K scratch owned by the library, for callers that cannot allocate device
+// memory themselves.  It lives in every device that loads this library, for
+// the life of the process.  Host code must not use the array's name as a device
+// address: the address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_decode_scratch[PA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+constexpr int kMaxScratchDevices = 128;
+std::mutex g_scratch_mutex;
+void *g_scratch_ptr[kMaxScratchDevices] = {};
+
+// Address of this device's copy of g_decode_scratch; looked up once per device
+// (with that device current) and cached.
+void *scratch_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return nullptr;
+    g_scratch_ptr[dev] = ptr;
+  }
+  return g_scratch_ptr[dev];
+}
+}  // namespace
+
+pa_status_t pa_decode_static_workspace(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                       const int32_t *block_tables, int max_blocks_per_seq,
+                                       const int32_t *context_lens, int num_seqs, int num_heads,
+                                       int max_context_len, float scale, int partition_size, int64_t num_blocks,
+                                       int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype,
+                                       void *stream) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_SHAPE;
+  const int P = resolve_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                       partition_size);
+  if (P <= 0) return PA_ERR_SHAPE;
+  const size_t need = workspace_layout(num_seqs, num_heads, head_dim, max_partitions(max_context_len, P)).bytes;
+  if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_WORKSPACE;
+  void *scratch = scratch_for_current_device();
+  if (!scratch) return PA_ERR_CUDA;
+  return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                   max_context_len, scale, partition_size, scratch, PA_STATIC_WORKSPACE_BYTES, num_blocks,
+                   block_size, num_kv_heads, head_dim, dtype, stream);
+}
+
 int pa_get_device_error(void *stream, int64_t *detail, int clear) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return -1;
   int code = 0;
