@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "pa.h"
 #include "pa_cache_ops.cuh"
@@ -61,8 +62,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // The cache [NB][16][Hkv][256 B] seen as a 5-D byte tensor
-// {128 B, 2 halves, Hkv, 16 tokens, NB}; the box is one (block, KV head) tile:
-// {128, 2, 1, 16, 1} = 4 KiB, landing 128-byte swizzled.
+// {128 B, 2 halves, Hkv, 16 tokens, NB}; the box is one half of one
+// (block, KV head) tile: {128, 1, 1, 16, 1} = 2 KiB (16 rows of 128 B),
+// landing 128-byte swizzled.  Two boxes make the 4 KiB tile.
 bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int num_kv_heads) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -70,7 +72,7 @@ bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, i
                               (cuuint64_t)num_blocks};
   const cuuint64_t strides[4] = {128, (cuuint64_t)kRowBytes, (cuuint64_t)num_kv_heads * kRowBytes,
                                  (cuuint64_t)kBlockSize * num_kv_heads * kRowBytes};
-  const cuuint32_t box[5] = {128, kRowBytes / 128, 1, kBlockSize, 1};
+  const cuuint32_t box[5] = {128, 1, 1, kBlockSize, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(cache), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -114,11 +116,11 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int 
   return w;
 }
 
-template <typename T, int G>
+template <typename T, int G, typename Math>
 pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
                           cudaStream_t stream) {
-  using SM = pa::DecodeSmem<T, G>;
-  auto kernel = pa::pa_decode_partition_kernel<T, G>;
+  using SM = pa::DecodeSmem<T, G, Math>;
+  auto kernel = pa::pa_decode_partition_kernel<T, G, Math>;
   // the attribute is per device; setting it on every call costs ~a microsecond of host time
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
     return PA_ERR_CUDA;
@@ -133,14 +135,23 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
   return launch_status();
 }
 
+// fp32 caches and single-head groups run on the CUDA cores; 16-bit caches with
+// grouped heads run the tensor-core block math.
 template <typename T>
 pa_status_t dispatch_group(int group, const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
                            cudaStream_t s) {
+  constexpr bool kMma = !std::is_same<T, float>::value;
   switch (group) {
-    case 1: return launch_decode<T, 1>(mk, mv, p, s);
-    case 2: return launch_decode<T, 2>(mk, mv, p, s);
-    case 4: return launch_decode<T, 4>(mk, mv, p, s);
-    case 8: return launch_decode<T, 8>(mk, mv, p, s);
+    case 1: return launch_decode<T, 1, pa::FmaMath<T, 1>>(mk, mv, p, s);
+    case 2:
+      if constexpr (kMma) return launch_decode<T, 2, pa::MmaMath<T, 2>>(mk, mv, p, s);
+      else return launch_decode<T, 2, pa::FmaMath<T, 2>>(mk, mv, p, s);
+    case 4:
+      if constexpr (kMma) return launch_decode<T, 4, pa::MmaMath<T, 4>>(mk, mv, p, s);
+      else return launch_decode<T, 4, pa::FmaMath<T, 4>>(mk, mv, p, s);
+    case 8:
+      if constexpr (kMma) return launch_decode<T, 8, pa::MmaMath<T, 8>>(mk, mv, p, s);
+      else return launch_decode<T, 8, pa::FmaMath<T, 8>>(mk, mv, p, s);
   }
   return PA_ERR_SHAPE;
 }

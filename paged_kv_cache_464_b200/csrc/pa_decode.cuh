@@ -13,40 +13,60 @@
 //   [p*P, min((p+1)*P, L_b)) of one KV head, serving all G = Hq/Hkv query heads
 //   of that KV head from a single read of each K/V block.  Sequences longer
 //   than P are split (split-K); each piece leaves an unnormalised partial
-//   (running max m, sum l, vector o) in the workspace and reduce_kernel
+//   (running max m, sum l, vector o) in the workspace and the reduce kernel
 //   combines them.  A sequence that fits in one partition is finished here.
 //
-// Inside a CTA (4 warps, no producer warp)
-//   Warp w owns the partition's blocks w, w+4, w+8, ... and keeps its own
+// Inside a CTA (kDecodeWarps warps, no producer warp)
+//   Warp w owns the partition's blocks w, w+W, w+2W, ... and keeps its own
 //   online-softmax state.  Each warp has kStagesPerWarp shared-memory stages;
 //   one elected lane issues a TMA tensor load for the K tile and the V tile of
-//   a block (16 tokens x 256 B each, a strided box of the [NB][16][Hkv][256 B]
-//   cache) into a stage, completing on that stage's mbarrier.  After a warp has
+//   a block into a stage, completing on that stage's mbarrier.  After a warp has
 //   used a stage it issues the load of its block kStagesPerWarp ahead into it.
-//   The tiles land 128-byte swizzled: the 16-byte chunk c of 128-byte row r
-//   sits at chunk position c ^ (r & 7), so the per-lane row reads below are
-//   free of bank conflicts.
+//   A tile is the 16 tokens x 256 B of one (block, KV head): a strided box of
+//   the cache, landing as [half][token][128 B] (half = which 128-byte half of
+//   the row) with the 128-byte swizzle: 16-byte chunk c of row r = half*16 + t
+//   sits at chunk position c ^ (t & 7).  Eight consecutive tokens therefore
+//   cover all 32 banks, so the row-per-lane reads (CUDA-core path) and the
+//   8x8 ldmatrix reads (tensor-core path) are free of bank conflicts.
 //
-//   QK: lane = 128-byte row r (token t = r / 2, half = r & 1 of the 256-byte
-//   row).  Each lane dots its half-row with the G query vectors (fp32,
-//   pre-scaled by scale*log2(e), broadcast from shared memory) with packed
-//   fp32x2 FMAs; one xor-shuffle joins the halves.
-//   Softmax: block max by a single warp reduction per head (redux.sync.max.f32),
-//   base-2 exponentials, running max/sum per warp (online softmax).
-//   PV: lane = (16-byte chunk cc of the output row, token parity); each lane
-//   accumulates G x (8 or 4) outputs over the block's tokens of its parity.
-//   Rows past the sequence end are skipped in PV (they may hold anything) and
-//   get weight 0 in QK.
-//   Epilogue: parities and warps are merged through shared memory.
+// Two ways to do a block's arithmetic (the pipeline is the same):
+//   FmaMath (fp32 caches, and G = 1): CUDA cores.  QK: lane = (token, half);
+//     each lane dots its half row with the G query vectors (fp32, pre-scaled
+//     by scale*log2(e), broadcast from shared memory) with packed fp32x2 FMAs,
+//     one shuffle joins the halves.  PV: lane = (output chunk, token parity).
+//   MmaMath (fp16/bf16 caches, G = 2..8): warp-level tensor-core MMA
+//     (m16n8k16, fp32 accumulate) on the transposed problem, so the G heads
+//     are the narrow N = 8 side and tokens / head_dim are the M = 16 side:
+//       S^T[16 tok][8 heads] = K[16 tok][128] . Q^T[128][8 heads]
+//       O^T[128][8 heads]   += V^T[128][16 tok] . P^T[16 tok][8 heads]
+//     K and V^T fragments come straight from the swizzled tiles (ldmatrix,
+//     .trans for V); Q^T fragments stay in registers for the whole partition;
+//     the S^T accumulator becomes the P^T operand with one 8x8 transpose
+//     (movmatrix) per 8 tokens.  P is fed as hi + lo 16-bit parts (two MMAs)
+//     so that rounding P to 16 bits costs nothing measurable (~2^-17).
+//   Both use base-2 online softmax with fp32 running max and sum.  Rows past
+//   the sequence end get weight 0 and never reach a multiply (their V rows
+//   may hold anything).
 #pragma once
 
 #include "pa_common.cuh"
 
 namespace pa {
 
-constexpr int kDecodeWarps = 4;
+// Launch shape (compile-time): warps per CTA, shared-memory stages per warp and
+// the CTAs per SM the register budget is sized for.
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES_PER_WARP
+#define PA_DECODE_STAGES_PER_WARP 2
+#endif
+#ifndef PA_DECODE_MIN_CTAS_PER_SM
+#define PA_DECODE_MIN_CTAS_PER_SM 3
+#endif
+constexpr int kDecodeWarps = PA_DECODE_WARPS;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
-constexpr int kStagesPerWarp = 2;
+constexpr int kStagesPerWarp = PA_DECODE_STAGES_PER_WARP;
 constexpr int kStages = kDecodeWarps * kStagesPerWarp;
 
 struct DecodeParams {
@@ -63,16 +83,374 @@ struct DecodeParams {
   float scale_log2;               // scale * log2(e)
 };
 
+// Byte offset of 16-byte chunk `c` (0..15) of token `t` in a swizzled tile.
+__device__ __forceinline__ int tile_offset(int t, int c) {
+  return ((c >> 3) * kBlockSize + t) * 128 + (((c & 7) ^ (t & 7)) << 4);
+}
+
+// ============================================================ CUDA-core math
 template <typename T, int G>
+struct FmaMath {
+  static constexpr int EPC = Elem<T>::kPerChunk;   // elements per 16-byte chunk
+  static constexpr int D = kChunksPerRow * EPC;
+  static constexpr int HALF = D / 2;
+  static constexpr int QS = HALF + 4;              // q row half stride (floats): halves on different banks
+  static constexpr int kQBytes = G * 2 * QS * 4;
+  static constexpr int kPBytes = kDecodeWarps * kBlockSize * G * 4;
+  static constexpr int kScratchBytes = kQBytes + kPBytes;
+  static constexpr bool kNeedsQInSmem = true;
+
+  float m_run[G], l_run[G];
+  float2 o[G][EPC / 2];
+  const float *q_s;
+  float *p_w;
+
+  // stage the G query vectors (fp32, pre-scaled, halves padded apart); CTA-wide
+  __device__ static void stage_q(uint8_t *scratch, const T *qg, float scale_log2) {
+    float *q_s = reinterpret_cast<float *>(scratch);
+    for (int i = threadIdx.x; i < G * D; i += kDecodeThreads) {
+      const int hh = i / D, d = i % D;
+      q_s[(hh * 2 + d / HALF) * QS + d % HALF] = Elem<T>::load(qg + i) * scale_log2;
+    }
+  }
+
+  __device__ void init(uint8_t *scratch, const T *, float, int warp, int) {
+    q_s = reinterpret_cast<const float *>(scratch);
+    p_w = reinterpret_cast<float *>(scratch + kQBytes) + warp * kBlockSize * G;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      m_run[hh] = -INFINITY;
+      l_run[hh] = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPC / 2; ++e) o[hh][e] = make_float2(0.f, 0.f);
+    }
+  }
+
+  __device__ void block(const uint8_t *tk, uint8_t *tv, int nvalid, int lane, float) {
+    // ---- scores of this lane's token (half row) for the G heads
+    const int t = lane & 15, half = lane >> 4;
+    float2 acc[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) acc[hh] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(tk + tile_offset(t, half * 8 + c));
+      float kf[EPC];
+      Elem<T>::unpack(raw, kf);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const float *qp = q_s + (hh * 2 + half) * QS + c * EPC;
+#pragma unroll
+        for (int e = 0; e < EPC; e += 4) {
+          const float4 qv = *reinterpret_cast<const float4 *>(qp + e);
+          acc[hh] = __ffma2_rn(make_float2(kf[e], kf[e + 1]), make_float2(qv.x, qv.y), acc[hh]);
+          acc[hh] = __ffma2_rn(make_float2(kf[e + 2], kf[e + 3]), make_float2(qv.z, qv.w), acc[hh]);
+        }
+      }
+    }
+    const bool valid = t < nvalid;
+    float pr[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      float sc = acc[hh].x + acc[hh].y;
+      sc += __shfl_xor_sync(kFullMask, sc, 16);
+      sc = valid ? sc : -INFINITY;
+      const float m_new = fmaxf(m_run[hh], warp_max(sc));
+      if (m_new != m_run[hh]) {   // warp-uniform
+        const float alpha = ex2(m_run[hh] - m_new);
+        l_run[hh] *= alpha;
+#pragma unroll
+        for (int e = 0; e < EPC / 2; ++e) o[hh][e] = __fmul2_rn(o[hh][e], make_float2(alpha, alpha));
+        m_run[hh] = m_new;
+      }
+      pr[hh] = ex2(sc - m_new);
+      l_run[hh] += pr[hh];
+    }
+    if (half == 0) {
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) p_w[t * G + hh] = pr[hh];
+    }
+    __syncwarp();
+
+    // ---- o += p * V over this lane's token parity
+    const int cc = lane & 15, par = lane >> 4;
+#pragma unroll
+    for (int i = 0; i < kBlockSize / 2; ++i) {
+      const int tt = 2 * i + par;
+      if (tt < nvalid) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(tv + tile_offset(tt, cc));
+        float vf[EPC];
+        Elem<T>::unpack(raw, vf);
+        float pv[G];
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int hh = 0; hh < G; hh += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(p_w + tt * G + hh);
+            pv[hh] = x.x; pv[hh + 1] = x.y; pv[hh + 2] = x.z; pv[hh + 3] = x.w;
+          }
+        } else if constexpr (G == 2) {
+          const float2 x = *reinterpret_cast<const float2 *>(p_w + tt * 2);
+          pv[0] = x.x; pv[1] = x.y;
+        } else {
+          pv[0] = p_w[tt];
+        }
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+          for (int e = 0; e < EPC / 2; ++e)
+            o[hh][e] = __ffma2_rn(make_float2(vf[2 * e], vf[2 * e + 1]), make_float2(pv[hh], pv[hh]), o[hh][e]);
+      }
+    }
+  }
+
+  // Merge the lane partials and write this warp's (m, l, o) for the G heads.
+  __device__ void write_partials(float *o_s, float *m_s, float *l_s, int warp, int lane) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      float l = l_run[hh];   // lanes t and t+16 hold the same p: sum over one half
+      l += __shfl_xor_sync(kFullMask, l, 1);
+      l += __shfl_xor_sync(kFullMask, l, 2);
+      l += __shfl_xor_sync(kFullMask, l, 4);
+      l += __shfl_xor_sync(kFullMask, l, 8);
+      l_run[hh] = l;
+#pragma unroll
+      for (int e = 0; e < EPC / 2; ++e) {
+        o[hh][e].x += __shfl_xor_sync(kFullMask, o[hh][e].x, 16);
+        o[hh][e].y += __shfl_xor_sync(kFullMask, o[hh][e].y, 16);
+      }
+    }
+    if (lane < 16) {
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int e = 0; e < EPC / 2; ++e)
+          *reinterpret_cast<float2 *>(o_s + (warp * G + hh) * D + lane * EPC + 2 * e) = o[hh][e];
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        m_s[warp * G + hh] = m_run[hh];
+        l_s[warp * G + hh] = l_run[hh];
+      }
+    }
+  }
+};
+
+// ============================================================ tensor-core math
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void *p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+template <typename T>
+struct MmaType;
+template <>
+struct MmaType<__nv_bfloat16> {
+  __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  // pack (lo, hi) into one register, rounding to nearest even; also return what was kept
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi, float &klo, float &khi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    const uint32_t u = *reinterpret_cast<uint32_t *>(&v);
+    klo = __uint_as_float(u << 16);
+    khi = __uint_as_float(u & 0xffff0000u);
+    return u;
+  }
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+  }
+};
+template <>
+struct MmaType<__half> {
+  __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi, float &klo, float &khi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    const float2 k = __half22float2(v);
+    klo = k.x;
+    khi = k.y;
+    return *reinterpret_cast<uint32_t *>(&v);
+  }
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+  }
+};
+
+template <typename T, int G>
+struct MmaMath {
+  static_assert(G >= 2 && G <= 8, "the N = 8 side holds up to 8 query heads");
+  static constexpr int D = 128;
+  static constexpr int kScratchBytes = 0;
+  static constexpr bool kNeedsQInSmem = false;
+
+  // Fragment roles (m16n8k16): gid = lane / 4 is the row group, tig = lane % 4.
+  //   S^T / P^T: this lane holds tokens gid and gid+8 for heads 2*tig, 2*tig+1.
+  //   O^T:       this lane holds d = 16*m + gid (+8) for heads 2*tig, 2*tig+1.
+  uint32_t qf[8][2];    // Q^T fragments, one pair per 16-wide k-step of head_dim
+  float m_run[2], l_run[2];
+  float o[8][4];        // O^T accumulators, 8 m-tiles of 16 d
+  int k_off[8];         // this lane's ldmatrix row address offsets for the K tile
+  int v_off[8];         // ... and for the V tile
+
+  __device__ static void stage_q(uint8_t *, const T *, float) {}
+
+  __device__ void init(uint8_t *, const T *qg, float, int, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (gid < G) {
+        const uint32_t *row = reinterpret_cast<const uint32_t *>(qg + gid * D + 16 * c + 2 * tig);
+        qf[c][0] = row[0];
+        qf[c][1] = row[4];   // + 8 elements
+      } else {
+        qf[c][0] = qf[c][1] = 0u;   // padding heads: zero query
+      }
+    }
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+    // ldmatrix: thread i addresses row (i % 8) of matrix (i / 8)
+    const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      // K as the A operand of k-step c: matrices (t0-7, d lo), (t8-15, d lo), (t0-7, d hi), (t8-15, d hi)
+      k_off[c] = tile_offset(ri + 8 * (mi & 1), 2 * c + (mi >> 1));
+      // V^T as the A operand of m-tile c: (t0-7, d lo), (t0-7, d hi), (t8-15, d lo), (t8-15, d hi), transposed
+      v_off[c] = tile_offset(ri + 8 * (mi >> 1), 2 * c + (mi & 1));
+    }
+  }
+
+  __device__ void block(const uint8_t *tk, uint8_t *tv, int nvalid, int lane, float scale_log2) {
+    const int gid = lane >> 2;
+    // ---- S^T = K Q^T for the block's 16 tokens
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t a[4];
+      ldmatrix_x4(a, tk + k_off[c]);
+      MmaType<T>::mma(s, a, qf[c][0], qf[c][1]);
+    }
+    const bool v0 = gid < nvalid, v1 = gid + 8 < nvalid;
+    const float x0 = v0 ? s[0] * scale_log2 : -INFINITY;
+    const float x1 = v0 ? s[1] * scale_log2 : -INFINITY;
+    const float x2 = v1 ? s[2] * scale_log2 : -INFINITY;
+    const float x3 = v1 ? s[3] * scale_log2 : -INFINITY;
+    // block max per head over the 16 tokens (lanes with equal tig)
+    float mb0 = fmaxf(x0, x2), mb1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mb0 = fmaxf(mb0, __shfl_xor_sync(kFullMask, mb0, off));
+      mb1 = fmaxf(mb1, __shfl_xor_sync(kFullMask, mb1, off));
+    }
+    const float mn0 = fmaxf(m_run[0], mb0), mn1 = fmaxf(m_run[1], mb1);
+    if (__any_sync(kFullMask, mn0 != m_run[0] || mn1 != m_run[1])) {
+      const float a0 = ex2(m_run[0] - mn0), a1 = ex2(m_run[1] - mn1);
+      l_run[0] *= a0;
+      l_run[1] *= a1;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        o[m][0] *= a0;
+        o[m][1] *= a1;
+        o[m][2] *= a0;
+        o[m][3] *= a1;
+      }
+      m_run[0] = mn0;
+      m_run[1] = mn1;
+    }
+    const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1), p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
+    l_run[0] += p0 + p2;
+    l_run[1] += p1 + p3;
+
+    // rows past the end hold anything: zero them so that 0 * V stays 0
+    if (nvalid < kBlockSize) {
+      uint4 *rows = reinterpret_cast<uint4 *>(tv);
+      const int n = (kBlockSize - nvalid) * 8;   // 16-byte chunks per half
+      for (int i = lane; i < 2 * n; i += 32) {
+        const int half = i / n, k = i % n;
+        rows[half * kBlockSize * 8 + nvalid * 8 + k] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
+    }
+
+    // ---- P^T fragments: hi and lo 16-bit parts, transposed from the S^T layout
+    float k0, k1, k2, k3;
+    const uint32_t h01 = MmaType<T>::pack(p0, p1, k0, k1);
+    const uint32_t h23 = MmaType<T>::pack(p2, p3, k2, k3);
+    const uint32_t l01 = MmaType<T>::pack(p0 - k0, p1 - k1);
+    const uint32_t l23 = MmaType<T>::pack(p2 - k2, p3 - k3);
+    const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+    const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+
+    // ---- O^T += V^T P^T
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(a, tv + v_off[m]);
+      MmaType<T>::mma(o[m], a, bh0, bh1);
+      MmaType<T>::mma(o[m], a, bl0, bl1);
+    }
+  }
+
+  __device__ void write_partials(float *o_s, float *m_s, float *l_s, int warp, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float l = l_run[j];   // sum over the 8 lanes that hold other tokens of the same heads
+      l += __shfl_xor_sync(kFullMask, l, 4);
+      l += __shfl_xor_sync(kFullMask, l, 8);
+      l += __shfl_xor_sync(kFullMask, l, 16);
+      l_run[j] = l;
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int hh = 2 * tig + j;
+      if (hh < G) {
+        float *dst = o_s + (warp * G + hh) * D + gid;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          dst[16 * m] = o[m][j];
+          dst[16 * m + 8] = o[m][2 + j];
+        }
+        if (gid == 0) {
+          m_s[warp * G + hh] = m_run[j];
+          l_s[warp * G + hh] = l_run[j];
+        }
+      }
+    }
+  }
+};
+
+// ============================================================ shared memory plan
+template <typename T, int G, typename Math>
 struct DecodeSmem {
-  static constexpr int kPerChunk = Elem<T>::kPerChunk;
-  static constexpr int D = kChunksPerRow * kPerChunk;
-  static constexpr int kHalf = D / 2;
-  static constexpr int kQStride = kHalf + 4;   // floats; pads the two halves onto different banks
+  static constexpr int D = kChunksPerRow * Elem<T>::kPerChunk;
   static constexpr int kTilesBytes = kStages * 2 * kTileBytes;
-  static constexpr int kQOff = kTilesBytes;
-  static constexpr int kPOff = kQOff + G * 2 * kQStride * 4;
-  static constexpr int kMOff = kPOff + kDecodeWarps * kBlockSize * G * 4;
+  static constexpr int kScratchOff = kTilesBytes;
+  static constexpr int kMOff = kScratchOff + Math::kScratchBytes;
   static constexpr int kLOff = kMOff + kDecodeWarps * G * 4;
   static constexpr int kFlagOff = kLOff + kDecodeWarps * G * 4;
   static constexpr int kBarOff = (kFlagOff + 4 + 7) / 8 * 8;
@@ -81,20 +459,17 @@ struct DecodeSmem {
   static_assert(kDecodeWarps * G * D * 4 <= kTilesBytes, "epilogue buffer must fit in the stage tiles");
 };
 
-template <typename T, int G>
-__global__ void __launch_bounds__(kDecodeThreads, 3)
+// ============================================================ partition kernel
+template <typename T, int G, typename Math>
+__global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
     pa_decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                const DecodeParams p) {
-  using SM = DecodeSmem<T, G>;
-  constexpr int EPC = SM::kPerChunk;
+  using SM = DecodeSmem<T, G, Math>;
   constexpr int D = SM::D;
-  constexpr int HALF = SM::kHalf;
-  constexpr int QS = SM::kQStride;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float *q_s = reinterpret_cast<float *>(smem + SM::kQOff);
-  float *p_s = reinterpret_cast<float *>(smem + SM::kPOff);
+  uint8_t *scratch = smem + SM::kScratchOff;
   float *m_s = reinterpret_cast<float *>(smem + SM::kMOff);
   float *l_s = reinterpret_cast<float *>(smem + SM::kLOff);
   int *abort_s = reinterpret_cast<int *>(smem + SM::kFlagOff);
@@ -127,6 +502,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3)
   const int tok0 = part * P;
   const int tok1 = min(tok0 + P, L);
   const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;
+  const T *qg = reinterpret_cast<const T *>(p.q) + (static_cast<size_t>(b) * p.num_heads + h0) * D;
 
   if (threadIdx.x == 0) {
     prefetch_tensor_map(&tm_k);
@@ -136,7 +512,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3)
     *abort_s = 0;
   }
 
-  // ---- this warp's blocks: local block index lb = warp + j * 4, j = 0 .. nw-1
+  // ---- this warp's blocks: local block index warp + j * W, j = 0 .. nw-1
   const int nw = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
   const int32_t *bt_row = p.block_tables + static_cast<size_t>(b) * p.max_blocks_per_seq + tok0 / kBlockSize;
   int id_group = -1;   // which 32 consecutive j's the lanes' ids belong to
@@ -158,47 +534,26 @@ __global__ void __launch_bounds__(kDecodeThreads, 3)
     const int s = warp + (j % kStagesPerWarp) * kDecodeWarps;
     if (lane == 0) {
       if (id >= 0) {
+        // one box per 128-byte half of the rows: the tile lands as [half][token][128 B]
         uint8_t *tk = smem + s * 2 * kTileBytes;
         mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
         tma_load_5d(tk, &tm_k, 0, 0, g, 0, id, &full[s], policy);
+        tma_load_5d(tk + kTileBytes / 2, &tm_k, 0, 1, g, 0, id, &full[s], policy);
         tma_load_5d(tk + kTileBytes, &tm_v, 0, 0, g, 0, id, &full[s], policy);
+        tma_load_5d(tk + kTileBytes + kTileBytes / 2, &tm_v, 0, 1, g, 0, id, &full[s], policy);
       } else {
         mbar_arrive(&full[s]);   // bad id: recorded above; complete the phase without data
       }
     }
   };
 
-  // query vectors of the G heads, fp32, pre-scaled, halves padded apart
-  {
-    const T *qg = reinterpret_cast<const T *>(p.q) + (static_cast<size_t>(b) * p.num_heads + h0) * D;
-    for (int i = threadIdx.x; i < G * D; i += kDecodeThreads) {
-      const int hh = i / D, d = i % D;
-      q_s[(hh * 2 + d / HALF) * QS + d % HALF] = Elem<T>::load(qg + i) * p.scale_log2;
-    }
-  }
-  __syncthreads();   // barriers initialised, q staged
+  if constexpr (Math::kNeedsQInSmem) Math::stage_q(scratch, qg, p.scale_log2);
+  __syncthreads();   // barriers initialised (and q staged)
 
   for (int j = 0; j < min(nw, kStagesPerWarp); ++j) issue(j);
 
-  float m_run[G], l_run[G];
-  float2 o[G][EPC / 2];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    m_run[hh] = -INFINITY;
-    l_run[hh] = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPC / 2; ++e) o[hh][e] = make_float2(0.f, 0.f);
-  }
-
-  // lane roles
-  const int r = lane;              // QK: 128-byte row of the tile
-  const int t_qk = r >> 1;         // its token
-  const int half = r & 1;          // which half of the 256-byte row
-  const int cc = lane & 15;        // PV: output chunk
-  const int par = lane >> 4;       // PV: token parity
-  const int r_pv_hi = cc >> 3;     // which 128-byte half holds chunk cc
-  const int c_pv = cc & 7;
-  float *p_w = p_s + warp * kBlockSize * G;
+  Math math;
+  math.init(scratch, qg, p.scale_log2, warp, lane);
 
   bool ok = true;
   int j = 0;
@@ -213,85 +568,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3)
       ok = false;
       break;
     }
-    const uint8_t *tk = smem + s * 2 * kTileBytes;
-    const uint8_t *tv = tk + kTileBytes;
+    uint8_t *tk = smem + s * 2 * kTileBytes;
     const int nvalid = min(kBlockSize, tok1 - (tok0 + (warp + j * kDecodeWarps) * kBlockSize));
-
-    // ---- scores of this lane's token for the G heads (half row each)
-    float2 acc[G];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) acc[hh] = make_float2(0.f, 0.f);
-    const uint8_t *krow = tk + r * 128;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(krow + ((c ^ (r & 7)) << 4));
-      float kf[EPC];
-      Elem<T>::unpack(raw, kf);
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float *qp = q_s + (hh * 2 + half) * QS + c * EPC;
-#pragma unroll
-        for (int e = 0; e < EPC; e += 4) {
-          const float4 qv = *reinterpret_cast<const float4 *>(qp + e);
-          acc[hh] = __ffma2_rn(make_float2(kf[e], kf[e + 1]), make_float2(qv.x, qv.y), acc[hh]);
-          acc[hh] = __ffma2_rn(make_float2(kf[e + 2], kf[e + 3]), make_float2(qv.z, qv.w), acc[hh]);
-        }
-      }
-    }
-    const bool valid = t_qk < nvalid;
-    float pr[G];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      float sc = acc[hh].x + acc[hh].y;
-      sc += __shfl_xor_sync(kFullMask, sc, 1);
-      sc = valid ? sc : -INFINITY;
-      const float m_new = fmaxf(m_run[hh], warp_max(sc));
-      if (m_new != m_run[hh]) {   // warp-uniform
-        const float alpha = ex2(m_run[hh] - m_new);
-        l_run[hh] *= alpha;
-#pragma unroll
-        for (int e = 0; e < EPC / 2; ++e) o[hh][e] = __fmul2_rn(o[hh][e], make_float2(alpha, alpha));
-        m_run[hh] = m_new;
-      }
-      pr[hh] = ex2(sc - m_new);
-      l_run[hh] += pr[hh];
-    }
-    if (half == 0) {
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) p_w[t_qk * G + hh] = pr[hh];
-    }
-    __syncwarp();
-
-    // ---- o += p * V over this lane's parity of the block's tokens
-#pragma unroll
-    for (int i = 0; i < kBlockSize / 2; ++i) {
-      const int tt = 2 * i + par;
-      if (tt < nvalid) {
-        const int rr = 2 * tt + r_pv_hi;
-        const uint4 raw = *reinterpret_cast<const uint4 *>(tv + rr * 128 + ((c_pv ^ (rr & 7)) << 4));
-        float vf[EPC];
-        Elem<T>::unpack(raw, vf);
-        float pv[G];
-        if constexpr (G % 4 == 0) {
-#pragma unroll
-          for (int hh = 0; hh < G; hh += 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(p_w + tt * G + hh);
-            pv[hh] = x.x; pv[hh + 1] = x.y; pv[hh + 2] = x.z; pv[hh + 3] = x.w;
-          }
-        } else if constexpr (G == 2) {
-          const float2 x = *reinterpret_cast<const float2 *>(p_w + tt * 2);
-          pv[0] = x.x; pv[1] = x.y;
-        } else {
-          pv[0] = p_w[tt];
-        }
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-          for (int e = 0; e < EPC / 2; ++e)
-            o[hh][e] = __ffma2_rn(make_float2(vf[2 * e], vf[2 * e + 1]), make_float2(pv[hh], pv[hh]), o[hh][e]);
-      }
-    }
-    __syncwarp();   // all lanes done with the stage and with p_w
+    math.block(tk, tk + kTileBytes, nvalid, lane, p.scale_log2);
+    __syncwarp();   // all lanes done with the stage
     if (j + kStagesPerWarp < nw) {
       fence_proxy_async_smem();
       issue(j + kStagesPerWarp);
@@ -303,37 +583,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3)
       mbar_wait(&full[warp + (jj % kStagesPerWarp) * kDecodeWarps], (jj / kStagesPerWarp) & 1);
   }
 
-  // ---- merge: l over the 16 tokens, o over the two parities
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    float l = l_run[hh];
-    l += __shfl_xor_sync(kFullMask, l, 2);
-    l += __shfl_xor_sync(kFullMask, l, 4);
-    l += __shfl_xor_sync(kFullMask, l, 8);
-    l += __shfl_xor_sync(kFullMask, l, 16);
-    l_run[hh] = l;
-#pragma unroll
-    for (int e = 0; e < EPC / 2; ++e) {
-      o[hh][e].x += __shfl_xor_sync(kFullMask, o[hh][e].x, 16);
-      o[hh][e].y += __shfl_xor_sync(kFullMask, o[hh][e].y, 16);
-    }
-  }
-  __syncthreads();   // every warp is done with the stage tiles: reuse them for the merge
+  // ---- merge the warps through shared memory (the stage tiles are reused)
+  __syncthreads();
   float *o_s = reinterpret_cast<float *>(smem);
-  if (par == 0) {
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-      for (int e = 0; e < EPC / 2; ++e)
-        *reinterpret_cast<float2 *>(o_s + (warp * G + hh) * D + cc * EPC + 2 * e) = o[hh][e];
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      m_s[warp * G + hh] = m_run[hh];
-      l_s[warp * G + hh] = l_run[hh];
-    }
-  }
+  math.write_partials(o_s, m_s, l_s, warp, lane);
   __syncthreads();
   if (*abort_s) return;
 
