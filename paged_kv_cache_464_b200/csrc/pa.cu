@@ -10,10 +10,15 @@
 #include <cstring>
 #include <mutex>
 #include <type_traits>
+#include <utility>
 
 #include "pa.h"
 #include "pa_cache_ops.cuh"
 #include "pa_decode.cuh"
+
+#ifndef PA_PROGRAMMATIC_LAUNCH
+#define PA_PROGRAMMATIC_LAUNCH 1
+#endif
 
 namespace {
 
@@ -41,8 +46,24 @@ pa_status_t cache_shape_status(int64_t num_blocks, int block_size, int num_kv_he
   return PA_OK;
 }
 
-pa_status_t launch_status() {
-  const cudaError_t e = cudaGetLastError();
+// Every kernel is launched with programmatic stream serialisation: it may be
+// scheduled while the previous kernel in the stream is still running, and it
+// waits (griddepcontrol.wait) before touching global memory, so stream order
+// semantics are unchanged while the launch latency overlaps the previous tail.
+template <typename... KArgs, typename... Args>
+pa_status_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                   Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = PA_PROGRAMMATIC_LAUNCH ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -81,17 +102,20 @@ bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, i
 }
 
 // ---------------------------------------------------------------- decode planning
+// Library choice of the partition size: 1024 tokens for the tensor-core block
+// math (16-bit caches, grouped heads), 512 for the CUDA-core one (measured best
+// on B200 for the GQA and MHA workloads); one partition when the longest
+// context fits.
 int resolve_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_context_len,
                            int requested) {
   (void)num_seqs;
-  (void)num_heads;
-  (void)num_kv_heads;
-  (void)head_dim;
-  if (max_context_len < 0 || requested < 0) return -1;
+  if (max_context_len < 0 || requested < 0 || num_kv_heads <= 0) return -1;
   if (requested > 0) return requested % kBlockSize == 0 ? requested : -1;
-  if (max_context_len <= 512) return max_context_len <= kBlockSize ? kBlockSize
-                                                                    : (max_context_len + kBlockSize - 1) / kBlockSize * kBlockSize;
-  return 512;
+  const bool tensor_core_math = head_dim == 128 && num_heads / num_kv_heads >= 2;
+  const int P = tensor_core_math ? 1024 : 512;
+  if (max_context_len <= P)
+    return max_context_len <= kBlockSize ? kBlockSize : (max_context_len + kBlockSize - 1) / kBlockSize * kBlockSize;
+  return P;
 }
 
 int max_partitions(int max_context_len, int partition_size) {
@@ -127,12 +151,12 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
   const long long grid = (long long)p.num_seqs * p.num_kv_heads * p.max_partitions;
   if (grid == 0) return PA_OK;
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
-  kernel<<<(unsigned)grid, pa::kDecodeThreads, SM::kAlloc, stream>>>(mk, mv, p);
-  pa_status_t st = launch_status();
+  pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(pa::kDecodeThreads), SM::kAlloc, stream, mk, mv, p);
   if (st != PA_OK || p.max_partitions <= 1) return st;
   const long long rows = (long long)p.num_seqs * p.num_heads;
-  pa::pa_decode_reduce_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
-  return launch_status();
+  if (rows > INT32_MAX) return PA_ERR_SHAPE;
+  constexpr int D = pa::kChunksPerRow * pa::Elem<T>::kPerChunk;
+  return launch(pa::pa_decode_reduce_kernel<T>, dim3((unsigned)rows), dim3(D), 0, stream, p);
 }
 
 // fp32 caches and single-head groups run on the CUDA cores; 16-bit caches with
@@ -176,10 +200,9 @@ pa_status_t pa_reshape_and_cache(const void *key, const void *value, void *k_cac
   const long long total = (long long)num_tokens * chunks_per_slot;
   long long blocks = (total + 255) / 256;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
-  pa::reshape_and_cache_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
-      (const uint4 *)key, (const uint4 *)value, (uint4 *)k_cache, (uint4 *)v_cache, slot_mapping, num_tokens,
-      chunks_per_slot, (long long)num_blocks * block_size);
-  return launch_status();
+  return launch(pa::reshape_and_cache_kernel, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream,
+                (const uint4 *)key, (const uint4 *)value, (uint4 *)k_cache, (uint4 *)v_cache, slot_mapping,
+                num_tokens, chunks_per_slot, (long long)num_blocks * block_size);
 }
 
 int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int max_context_len,
@@ -268,10 +291,9 @@ pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_ma
   if (!k_cache || !v_cache || !block_mapping) return PA_ERR_NULL;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8)) return PA_ERR_ALIGN;
   const int chunks_per_block = kBlockSize * num_kv_heads * (kRowBytes / 16);
-  pa::copy_blocks_kernel<<<dim3((unsigned)num_pairs, 2), 256, 0, (cudaStream_t)stream>>>(
-      (uint4 *)k_cache, (uint4 *)v_cache, (const long long *)block_mapping, num_pairs, (long long)num_blocks,
-      chunks_per_block);
-  return launch_status();
+  return launch(pa::copy_blocks_kernel, dim3((unsigned)num_pairs, 2), dim3(256), 0, (cudaStream_t)stream,
+                (uint4 *)k_cache, (uint4 *)v_cache, (const long long *)block_mapping, num_pairs,
+                (long long)num_blocks, chunks_per_block);
 }
 
 // ---------------------------------------------------------------- no-allocation decode

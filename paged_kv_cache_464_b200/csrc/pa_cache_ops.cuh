@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4 *__r
                                                                 const int64_t *__restrict__ slot_mapping,
                                                                 int num_tokens, int chunks_per_slot,
                                                                 long long num_slots) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = static_cast<long long>(num_tokens) * chunks_per_slot;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -44,6 +46,8 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ k_
                                                           const long long *__restrict__ block_mapping,
                                                           int num_pairs, long long num_blocks,
                                                           int chunks_per_block) {
+  pdl_wait();
+  pdl_trigger();
   const int pair = blockIdx.x;
   const long long src = block_mapping[2 * pair];
   const long long dst = block_mapping[2 * pair + 1];

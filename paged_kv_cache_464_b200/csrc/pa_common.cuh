@@ -108,6 +108,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- launch ordering
+// Programmatic dependent launch: kernels are launched so that the next kernel
+// in the stream may start before this one ends.  Each kernel calls pdl_wait()
+// before its first global-memory access (it returns once the previous grid in
+// the stream has completed and its writes are visible; a no-op when launched
+// without the attribute), and pdl_trigger() to let its successor launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2(float x) {   // 2^x; ex2(-inf) = +0
   float y;
@@ -142,6 +151,7 @@ struct Elem<float> {
   __device__ __forceinline__ static void store2(float *p, float a, float b) {
     *reinterpret_cast<float2 *>(p) = make_float2(a, b);
   }
+  __device__ __forceinline__ static void store1(float *p, float a) { *p = a; }
 };
 
 template <>
@@ -170,6 +180,7 @@ struct Elem<__nv_bfloat16> {
   __device__ __forceinline__ static void store2(__nv_bfloat16 *p, float a, float b) {
     *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
   }
+  __device__ __forceinline__ static void store1(__nv_bfloat16 *p, float a) { *p = __float2bfloat16_rn(a); }
 };
 
 template <>
@@ -197,6 +208,7 @@ struct Elem<__half> {
   __device__ __forceinline__ static void store2(__half *p, float a, float b) {
     *reinterpret_cast<__half2 *>(p) = __floats2half2_rn(a, b);
   }
+  __device__ __forceinline__ static void store1(__half *p, float a) { *p = __float2half_rn(a); }
 };
 
 }  // namespace pa

@@ -477,6 +477,8 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_wait();      // the previous kernel's writes (caches, inputs) are visible from here on
+  pdl_trigger();   // the reduce kernel may be scheduled once every CTA of this grid has started
 
   // ---- work item: blockIdx.x = ((b * Hkv) + g) * NPmax + part
   int item = blockIdx.x;
@@ -624,14 +626,15 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
 // Combine the partitions of every (sequence, query head) that was split:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
 // (m_p are base-2 log-domain maxima; o_p and l_p are relative to m_p).
-// One warp per (b, h); each lane owns D/32 consecutive outputs.
+// One CTA of D threads per (b, h) row; thread t owns output element t, so every
+// partition's partial vector is read as one coalesced row.
 template <typename T>
 __global__ void __launch_bounds__(128) pa_decode_reduce_kernel(const DecodeParams p) {
   constexpr int D = kChunksPerRow * Elem<T>::kPerChunk;
-  constexpr int PER_LANE = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-  if (row >= static_cast<long long>(p.num_seqs) * p.num_heads) return;
+  constexpr int kWarps = D / 32;
+  __shared__ float red_s[kWarps];
+  pdl_wait();   // the partition kernel's partials are visible from here on
+  const long long row = blockIdx.x;
   const int b = static_cast<int>(row / p.num_heads);
   const int L = p.context_lens[b];
   if (L < 0 || L > p.max_context_len || L > p.max_blocks_per_seq * kBlockSize) return;
@@ -639,45 +642,36 @@ __global__ void __launch_bounds__(128) pa_decode_reduce_kernel(const DecodeParam
   if (np <= 1) return;   // finished by the partition kernel
   const float *m = p.ws_m + row * p.max_partitions;
   const float *l = p.ws_l + row * p.max_partitions;
-  const float *o = p.ws_o + row * p.max_partitions * D;
+  const float *o = p.ws_o + row * p.max_partitions * D + threadIdx.x;
 
   float M = -INFINITY;
-  for (int i = lane; i < np; i += 32) M = fmaxf(M, m[i]);
+  for (int i = threadIdx.x; i < np; i += D) M = fmaxf(M, m[i]);
   M = warp_max(M);
-  float lsum = 0.f;
-  float acc[PER_LANE];
+  if ((threadIdx.x & 31) == 0) red_s[threadIdx.x >> 5] = M;
+  __syncthreads();
 #pragma unroll
-  for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
-  for (int base = 0; base < np; base += 32) {
-    const int i = base + lane;
-    const float w = i < np ? ex2(m[i] - M) : 0.f;
-    lsum += i < np ? w * l[i] : 0.f;
-    const int n = min(32, np - base);
-    for (int k = 0; k < n; ++k) {
-      const float wk = __shfl_sync(kFullMask, w, k);
-      const float *src = o + static_cast<size_t>(base + k) * D + lane * PER_LANE;
-      if constexpr (PER_LANE == 4) {
-        const float4 x = *reinterpret_cast<const float4 *>(src);
-        acc[0] += wk * x.x;
-        acc[1] += wk * x.y;
-        acc[2] += wk * x.z;
-        acc[3] += wk * x.w;
-      } else {
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red_s[w]);
+
+  float lsum = 0.f, acc = 0.f;
+  int i = 0;
+  for (; i + 8 <= np; i += 8) {
+    float x[8], w[8];
 #pragma unroll
-        for (int e = 0; e < PER_LANE; ++e) acc[e] += wk * src[e];
-      }
+    for (int k = 0; k < 8; ++k) x[k] = o[static_cast<size_t>(i + k) * D];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      w[k] = ex2(m[i + k] - M);
+      lsum += w[k] * l[i + k];
+      acc += w[k] * x[k];
     }
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, off);
-  const float inv = 1.f / lsum;
-  T *out = reinterpret_cast<T *>(p.out) + row * D + lane * PER_LANE;
-  if constexpr (PER_LANE == 4) {
-    Elem<T>::store4(out, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  } else {
-    static_assert(PER_LANE == 2, "D is 64 or 128");
-    Elem<T>::store2(out, acc[0] * inv, acc[1] * inv);
+  for (; i < np; ++i) {
+    const float w = ex2(m[i] - M);
+    lsum += w * l[i];
+    acc += w * o[static_cast<size_t>(i) * D];
   }
+  T *out = reinterpret_cast<T *>(p.out) + row * D + threadIdx.x;
+  Elem<T>::store1(out, acc / lsum);
 }
 
 }  // namespace pa
