@@ -189,26 +189,33 @@ class Step:
         ws = capi.decode_workspace_bytes(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, self.maxL, self.P)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
         self.has_pairs = case.block_mapping.numel() > 0
-        self.launches_per_step = self._count_launches()
 
-    def _count_launches(self):
+    def launches(self, fused: bool) -> int:
         c = self.case.cfg
         P = self.pa.decode_partition_size(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, self.maxL, self.P)
         split = math.ceil(self.maxL / P) > 1
-        return (1 if self.has_pairs else 0) + 1 + 1 + (1 if split else 0)
+        return (1 if self.has_pairs else 0) + (0 if fused else 1) + 1 + (1 if split else 0)
 
+    # fused step: copies, then the new-token write and decode in one launch (pa_decode_append)
     def pre(self):
         if self.has_pairs:
             self.pa.copy_blocks(self.k, self.v, self.pairs)
-        self.pa.reshape_and_cache(self.key, self.value, self.k, self.v, self.slots)
 
     def decode(self):
-        self.pa.decode(self.q, self.k, self.v, self.bt, self.cl, self.case.scale, out=self.out,
-                       max_context_len=self.maxL, partition_size=self.P, workspace=self.ws)
+        self.pa.decode_append(self.q, self.key, self.value, self.k, self.v, self.bt, self.cl, self.case.scale,
+                              out=self.out, max_context_len=self.maxL, partition_size=self.P, workspace=self.ws)
 
     def __call__(self):
         self.pre()
         self.decode()
+
+    # the same step as three separate calls (pa_copy_blocks, pa_reshape_and_cache, pa_decode)
+    def separate(self):
+        if self.has_pairs:
+            self.pa.copy_blocks(self.k, self.v, self.pairs)
+        self.pa.reshape_and_cache(self.key, self.value, self.k, self.v, self.slots)
+        self.pa.decode(self.q, self.k, self.v, self.bt, self.cl, self.case.scale, out=self.out,
+                       max_context_len=self.maxL, partition_size=self.P, workspace=self.ws)
 
 
 def run_ours(args, world, rank, local):
@@ -225,26 +232,47 @@ def run_ours(args, world, rank, local):
         step()
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps; decode launches bracketed by events for the roofline
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+    # ---- timed region: exactly K steps, events only at its two ends (an event
+    # between launches would stop the next kernel from being scheduled early)
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.time()
     t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t_start.elapsed_time(t_stop)
+
+    # ---- roofline pass: the same K steps with the decode launches bracketed by
+    # events on the launching stream, for the kernel's own average duration
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    torch.cuda.synchronize()
     for i in range(args.steps):
         step.pre()
         ev_dec[i][0].record(stream)
         step.decode()
         ev_dec[i][1].record(stream)
-    t_stop.record(stream)
     torch.cuda.synchronize()
-    wall1 = time.time()
-    barrier(world)
-    elapsed_ms = t_start.elapsed_time(t_stop)
     dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+
+    # the same K steps as three separate calls, for comparison
+    for _ in range(args.warmup):
+        step.separate()
+    s_start, s_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    s_start.record(stream)
+    for _ in range(args.steps):
+        step.separate()
+    s_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    sep_ms = s_start.elapsed_time(s_stop)
 
     # keep the GPU under the same load long enough for the clock sampler
     soak_until = wall0 + 1.5
@@ -259,6 +287,7 @@ def run_ours(args, world, rank, local):
     e2e = run_e2e(case, step, args.steps, args.warmup, device)
 
     max_ms = all_reduce_max(elapsed_ms, world, device)
+    sep_max_ms = all_reduce_max(sep_ms, world, device)
     total_bytes = all_reduce_sum(float(kv_bytes), world, device)
     total_seqs = all_reduce_sum(float(cfg.num_seqs), world, device)
     e2e_ms = all_reduce_max(e2e["ms"], world, device)
@@ -297,14 +326,18 @@ def run_ours(args, world, rank, local):
             "kv_bytes_per_step_per_gpu": kv_bytes,
             "partition_size": step.pa.decode_partition_size(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads,
                                                             cfg.head_dim, step.maxL, step.P),
-            "step": ("copy_blocks + " if step.has_pairs else "") + "reshape_and_cache + decode",
+            "step": ("pa_copy_blocks + " if step.has_pairs else "") + "pa_decode_append (new-token write + decode)",
             "l2": f"inputs larger than L2: {kv_bytes / 2**20:.0f} MiB of KV per step vs 126 MiB L2, no flush",
             "parallelism": f"replicas x{world}, no data-path collective",
         },
         "seqs_per_s": round(total_seqs * args.steps / (max_ms * 1e-3), 1),
+        "step_separate_calls": {
+            "calls": ("pa_copy_blocks + " if step.has_pairs else "") + "pa_reshape_and_cache + pa_decode",
+            "value": round(total_bytes * args.steps / (sep_max_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(sep_max_ms / args.steps, 5)},
         "pct_hbm_peak": round(100.0 * value / world / peak, 2),
         "roofline": {
-            "kernel": "pa_decode (partition + reduce launches)",
+            "kernel": "pa_decode_append (partition + reduce launches)",
             "bound": "hbm",
             "achieved": round(achieved, 2),
             "peak": peak,
@@ -319,7 +352,7 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": round(total_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "ms_per_step": round(e2e_ms / args.steps, 5)},
-        "gpu_launches": step.launches_per_step * args.steps,
+        "gpu_launches": step.launches(fused=True) * args.steps,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -148,6 +148,29 @@ pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void 
                       int head_dim, pa_dtype_t dtype, void *stream);
 
 /*
+ * pa_decode_append -- the decode step's new-token write and decode in one
+ * launch ([A] §五 PagedAttention.forward: the current token's k/v join the
+ * cache and are attended together with it; [A] §三 append_token: the token
+ * goes to the next offset of the sequence's last block).
+ *
+ * For every sequence with context_lens[b] >= 1, the new token is position
+ * L = context_lens[b] - 1: its K and V rows key[b] and value[b]
+ * ([num_seqs][num_kv_heads][head_dim], cache dtype) are written bit-exactly to
+ * row (block_tables[b][L / 16], L % 16) of k_cache / v_cache, and the sequence
+ * is then decoded over all context_lens[b] tokens exactly as pa_decode does.
+ * Same result as pa_reshape_and_cache with slot = block_tables[b][L/16]*16 +
+ * L%16 followed by pa_decode, in one kernel (plus the reduce when split).
+ * Arguments and errors are those of pa_decode plus key/value (non-NULL,
+ * 16-byte aligned); the caches are written, so they are not const here.
+ */
+pa_status_t pa_decode_append(void *out, const void *q, const void *key, const void *value, void *k_cache,
+                             void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len,
+                             float scale, int partition_size, void *workspace, size_t workspace_bytes,
+                             int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                             pa_dtype_t dtype, void *stream);
+
+/*
  * pa_copy_blocks -- copy-on-write block copies ([B] Block 管理器, item 3:
  * when a request writes to a block that several requests share, the block is
  * copied first and the request's table is pointed at the copy; the caller

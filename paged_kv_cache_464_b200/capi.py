@@ -28,6 +28,9 @@ _lib.pa_decode_workspace_bytes.restype = _SZ
 _lib.pa_decode_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.pa_decode.restype = _I
 _lib.pa_decode.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _P, _SZ, _I64, _I, _I, _I, _I, _P]
+_lib.pa_decode_append.restype = _I
+_lib.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _P, _SZ, _I64, _I, _I, _I,
+                                  _I, _P]
 _lib.pa_decode_static_workspace.restype = _I
 _lib.pa_decode_static_workspace.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _I64, _I, _I, _I, _I,
                                             _P]
@@ -39,7 +42,7 @@ _lib.pa_status_string.restype = ctypes.c_char_p
 _lib.pa_status_string.argtypes = [_I]
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_static_workspace", "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
+            "pa_decode_append", "pa_decode_static_workspace", "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
 STATIC_WORKSPACE_BYTES = 64 << 20   # PA_STATIC_WORKSPACE_BYTES in include/pa.h
 
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
@@ -144,6 +147,43 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
                           _dev(block_tables, "block_tables"), block_tables.shape[1],
                           _dev(context_lens, "context_lens"), S, hq, max_context_len, float(scale),
                           partition_size, ws_ptr, ws_bytes, nb, bs, hkv, d, dt, _stream(stream)), "pa_decode")
+    return out
+
+
+def decode_append(q: torch.Tensor, key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor,
+                  v_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                  out: Optional[torch.Tensor] = None, *, max_context_len: Optional[int] = None,
+                  partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Write each sequence's new token (key/value [S, Hkv, D]) at position
+    context_len - 1 through its block table, then decode -- one launch."""
+    nb, bs, hkv, d, dt = _cache_args(k_cache, v_cache)
+    S, hq, dq = q.shape
+    if dq != d or q.dtype != k_cache.dtype or key.dtype != k_cache.dtype or value.dtype != k_cache.dtype:
+        raise ValueError("q, key and value must have the cache dtype and head_dim")
+    if tuple(key.shape) != (S, hkv, d) or tuple(value.shape) != (S, hkv, d):
+        raise ValueError("key/value must be [S, num_kv_heads, head_dim]")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("block_tables must be [S, max_blocks_per_seq] and context_lens [S]")
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if S else 0
+    need = decode_workspace_bytes(S, hq, hkv, d, max_context_len, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pa_decode_append(_dev(out, "out"), _dev(q, "q"), _dev(key, "key"), _dev(value, "value"),
+                                 _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                 _dev(block_tables, "block_tables"), block_tables.shape[1],
+                                 _dev(context_lens, "context_lens"), S, hq, max_context_len, float(scale),
+                                 partition_size, ws_ptr, ws_bytes, nb, bs, hkv, d, dt, _stream(stream)),
+           "pa_decode_append")
     return out
 
 

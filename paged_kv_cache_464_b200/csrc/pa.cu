@@ -153,10 +153,11 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
   pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(pa::kDecodeThreads), SM::kAlloc, stream, mk, mv, p);
   if (st != PA_OK || p.max_partitions <= 1) return st;
+  // a fixed grid of warps walks all (sequence, head) rows: 8 CTAs of 4 warps per SM at most
   const long long rows = (long long)p.num_seqs * p.num_heads;
-  if (rows > INT32_MAX) return PA_ERR_SHAPE;
-  constexpr int D = pa::kChunksPerRow * pa::Elem<T>::kPerChunk;
-  return launch(pa::pa_decode_reduce_kernel<T>, dim3((unsigned)rows), dim3(D), 0, stream, p);
+  long long ctas = (rows + pa::kReduceWarps - 1) / pa::kReduceWarps;
+  if (ctas > 148LL * 8) ctas = 148LL * 8;
+  return launch(pa::pa_decode_reduce_kernel<T>, dim3((unsigned)ctas), dim3(pa::kReduceWarps * 32), 0, stream, p);
 }
 
 // fp32 caches and single-head groups run on the CUDA cores; 16-bit caches with
@@ -219,11 +220,15 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, 
   return workspace_layout(num_seqs, num_heads, head_dim, max_partitions(max_context_len, P)).bytes;
 }
 
-pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
-                      const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
-                      int num_seqs, int num_heads, int max_context_len, float scale, int partition_size,
-                      void *workspace, size_t workspace_bytes, int64_t num_blocks, int block_size,
-                      int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream) {
+}  // extern "C"
+
+namespace {
+
+pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void *new_v, const void *k_cache,
+                        const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                        const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len, float scale,
+                        int partition_size, void *workspace, size_t workspace_bytes, int64_t num_blocks,
+                        int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream) {
   pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 || max_blocks_per_seq < 0 ||
@@ -271,6 +276,10 @@ pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void 
   p.partition_size = P;
   p.max_partitions = np;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.new_k = new_k;
+  p.new_v = new_v;
+  p.k_cache = new_k ? const_cast<void *>(k_cache) : nullptr;
+  p.v_cache = new_k ? const_cast<void *>(v_cache) : nullptr;
 
   cudaStream_t s = (cudaStream_t)stream;
   switch (dtype) {
@@ -279,6 +288,33 @@ pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void 
     case PA_BF16: return dispatch_group<__nv_bfloat16>(group, mk, mv, p, s);
   }
   return PA_ERR_DTYPE;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                      int num_seqs, int num_heads, int max_context_len, float scale, int partition_size,
+                      void *workspace, size_t workspace_bytes, int64_t num_blocks, int block_size,
+                      int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream) {
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     num_seqs, num_heads, max_context_len, scale, partition_size, workspace, workspace_bytes,
+                     num_blocks, block_size, num_kv_heads, head_dim, dtype, stream);
+}
+
+pa_status_t pa_decode_append(void *out, const void *q, const void *key, const void *value, void *k_cache,
+                             void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len,
+                             float scale, int partition_size, void *workspace, size_t workspace_bytes,
+                             int64_t num_blocks, int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype,
+                             void *stream) {
+  if (num_seqs > 0 && (!key || !value)) return PA_ERR_NULL;
+  if (!aligned(key, 16) || !aligned(value, 16)) return PA_ERR_ALIGN;
+  return decode_impl(out, q, key, value, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     num_seqs, num_heads, max_context_len, scale, partition_size, workspace, workspace_bytes,
+                     num_blocks, block_size, num_kv_heads, head_dim, dtype, stream);
 }
 
 pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,

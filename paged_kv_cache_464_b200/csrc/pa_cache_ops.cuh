@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4 *__r
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
     const int tok = static_cast<int>(i / chunks_per_slot);
     const int rem = static_cast<int>(i - static_cast<long long>(tok) * chunks_per_slot);
+    const uint4 kx = key[i];   // issued before the slot load so the latencies overlap
+    const uint4 vx = value[i];
     const long long slot = slot_mapping[tok];
     if (slot < 0) continue;   // padding token: nothing to write
     if (slot >= num_slots) {
@@ -33,8 +35,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4 *__r
       continue;
     }
     const long long dst = slot * chunks_per_slot + rem;
-    k_cache[dst] = key[i];
-    v_cache[dst] = value[i];
+    k_cache[dst] = kx;
+    v_cache[dst] = vx;
   }
 }
 

@@ -81,6 +81,10 @@ struct DecodeParams {
   int num_seqs, num_heads, num_kv_heads, max_blocks_per_seq;
   int max_context_len, partition_size, max_partitions;
   float scale_log2;               // scale * log2(e)
+  // append mode (all non-null) or plain decode (all null): the step's new token
+  // rows [S][Hkv][D], written at position context_len - 1 before it is attended
+  const void *new_k, *new_v;
+  void *k_cache, *v_cache;
 };
 
 // Byte offset of 16-byte chunk `c` (0..15) of token `t` in a swizzled tile.
@@ -571,7 +575,28 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
       break;
     }
     uint8_t *tk = smem + s * 2 * kTileBytes;
-    const int nvalid = min(kBlockSize, tok1 - (tok0 + (warp + j * kDecodeWarps) * kBlockSize));
+    const int lb = warp + j * kDecodeWarps;   // local block index
+    const int nvalid = min(kBlockSize, tok1 - (tok0 + lb * kBlockSize));
+    if (p.new_k != nullptr && part == nparts - 1 && lb == nblk - 1) {
+      // append mode: this block holds position L-1.  Store the new token's K/V
+      // rows of head g in the cache and put them into the tile that just landed
+      // (its copy of that row may predate the store).  Lanes 0-15 move the 16
+      // chunks of the K row, lanes 16-31 those of the V row.
+      const int t_new = (L - 1) % kBlockSize;
+      const int c = lane & 15;
+      const bool is_v = lane >= 16;
+      const uint4 *src = reinterpret_cast<const uint4 *>(is_v ? p.new_v : p.new_k) +
+                         (static_cast<size_t>(b) * p.num_kv_heads + g) * kChunksPerRow + c;
+      const uint4 x = *src;
+      const int id = bt_row[lb];
+      if (id >= 0 && id < p.num_blocks) {
+        uint4 *dst = reinterpret_cast<uint4 *>(is_v ? p.v_cache : p.k_cache) +
+                     ((static_cast<size_t>(id) * kBlockSize + t_new) * p.num_kv_heads + g) * kChunksPerRow + c;
+        *dst = x;
+      }
+      *reinterpret_cast<uint4 *>(tk + (is_v ? kTileBytes : 0) + tile_offset(t_new, c)) = x;
+      __syncwarp();
+    }
     math.block(tk, tk + kTileBytes, nvalid, lane, p.scale_log2);
     __syncwarp();   // all lanes done with the stage
     if (j + kStagesPerWarp < nw) {
@@ -626,52 +651,81 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
 // Combine the partitions of every (sequence, query head) that was split:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
 // (m_p are base-2 log-domain maxima; o_p and l_p are relative to m_p).
-// One CTA of D threads per (b, h) row; thread t owns output element t, so every
-// partition's partial vector is read as one coalesced row.
+// A fixed grid of warps walks the (b, h) rows (rows that were not split are
+// skipped after one load); lane l owns outputs [l*D/32, (l+1)*D/32), so each
+// partition's partial vector is one coalesced row read.
+constexpr int kReduceWarps = 4;
+
 template <typename T>
-__global__ void __launch_bounds__(128) pa_decode_reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(const DecodeParams p) {
   constexpr int D = kChunksPerRow * Elem<T>::kPerChunk;
-  constexpr int kWarps = D / 32;
-  __shared__ float red_s[kWarps];
+  constexpr int PER_LANE = D / 32;
   pdl_wait();   // the partition kernel's partials are visible from here on
-  const long long row = blockIdx.x;
-  const int b = static_cast<int>(row / p.num_heads);
-  const int L = p.context_lens[b];
-  if (L < 0 || L > p.max_context_len || L > p.max_blocks_per_seq * kBlockSize) return;
-  const int np = (L + p.partition_size - 1) / p.partition_size;
-  if (np <= 1) return;   // finished by the partition kernel
-  const float *m = p.ws_m + row * p.max_partitions;
-  const float *l = p.ws_l + row * p.max_partitions;
-  const float *o = p.ws_o + row * p.max_partitions * D + threadIdx.x;
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(p.num_seqs) * p.num_heads;
+  const long long stride = static_cast<long long>(gridDim.x) * kReduceWarps;
+  for (long long row = static_cast<long long>(blockIdx.x) * kReduceWarps + (threadIdx.x >> 5); row < rows;
+       row += stride) {
+    const int b = static_cast<int>(row / p.num_heads);
+    const int L = p.context_lens[b];
+    if (L < 0 || L > p.max_context_len || L > p.max_blocks_per_seq * kBlockSize) continue;
+    const int np = (L + p.partition_size - 1) / p.partition_size;
+    if (np <= 1) continue;   // finished by the partition kernel
+    const float *m = p.ws_m + row * p.max_partitions;
+    const float *l = p.ws_l + row * p.max_partitions;
+    const float *o = p.ws_o + row * p.max_partitions * D + lane * PER_LANE;
 
-  float M = -INFINITY;
-  for (int i = threadIdx.x; i < np; i += D) M = fmaxf(M, m[i]);
-  M = warp_max(M);
-  if ((threadIdx.x & 31) == 0) red_s[threadIdx.x >> 5] = M;
-  __syncthreads();
+    float M = -INFINITY;
+    for (int i = lane; i < np; i += 32) M = fmaxf(M, m[i]);
+    M = warp_max(M);
+    float lsum = 0.f;
+    float acc[PER_LANE];
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red_s[w]);
-
-  float lsum = 0.f, acc = 0.f;
-  int i = 0;
-  for (; i + 8 <= np; i += 8) {
-    float x[8], w[8];
+    for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
+    for (int base = 0; base < np; base += 32) {
+      const int i = base + lane;
+      const float w = i < np ? ex2(m[i] - M) : 0.f;
+      lsum += i < np ? w * l[i] : 0.f;
+      const int n = min(32, np - base);
+      int k = 0;
+      for (; k + 4 <= n; k += 4) {   // four partials in flight
+        float x[4][PER_LANE];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) x[k] = o[static_cast<size_t>(i + k) * D];
+        for (int u = 0; u < 4; ++u) {
+          const float *src = o + static_cast<size_t>(base + k + u) * D;
+          if constexpr (PER_LANE == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(src);
+            x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2 *>(src);
+            x[u][0] = v.x; x[u][1] = v.y;
+          }
+        }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      w[k] = ex2(m[i + k] - M);
-      lsum += w[k] * l[i + k];
-      acc += w[k] * x[k];
+        for (int u = 0; u < 4; ++u) {
+          const float wk = __shfl_sync(kFullMask, w, k + u);
+#pragma unroll
+          for (int e = 0; e < PER_LANE; ++e) acc[e] += wk * x[u][e];
+        }
+      }
+      for (; k < n; ++k) {
+        const float wk = __shfl_sync(kFullMask, w, k);
+        const float *src = o + static_cast<size_t>(base + k) * D;
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) acc[e] += wk * src[e];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, off);
+    const float inv = 1.f / lsum;
+    T *out = reinterpret_cast<T *>(p.out) + row * D + lane * PER_LANE;
+    if constexpr (PER_LANE == 4) {
+      Elem<T>::store4(out, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    } else {
+      Elem<T>::store2(out, acc[0] * inv, acc[1] * inv);
     }
   }
-  for (; i < np; ++i) {
-    const float w = ex2(m[i] - M);
-    lsum += w * l[i];
-    acc += w * o[static_cast<size_t>(i) * D];
-  }
-  T *out = reinterpret_cast<T *>(p.out) + row * D + threadIdx.x;
-  Elem<T>::store1(out, acc / lsum);
 }
 
 }  // namespace pa

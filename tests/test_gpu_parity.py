@@ -248,3 +248,47 @@ def test_streams_and_repeat_determinism(pa):
         b = pa.decode(d["q"], k, v, d["bt"], d["cl"], case.scale, max_context_len=4000)
     s.synchronize()
     assert torch.equal(a.cpu(), b.cpu())
+
+
+def gpu_step_append(pa, case, partition_size=None):
+    """The step through the fused entry point: copies, then write + decode in one launch."""
+    d = to_dev(case)
+    if case.block_mapping.numel():
+        pa.copy_blocks(d["k"], d["v"], d["pairs"])
+    P = case.cfg.partition_size if partition_size is None else partition_size
+    out = pa.decode_append(d["q"], d["key"], d["value"], d["k"], d["v"], d["bt"], d["cl"], case.scale,
+                           max_context_len=case.max_context_len, partition_size=P)
+    torch.cuda.synchronize()
+    return out, d
+
+
+@pytest.mark.parametrize("name", list(inputs.CONFIGS))
+def test_append_step_small(pa, orc, name):
+    case = inputs.make_case(name, lens=SMALL[name])
+    out, d = gpu_step_append(pa, case)
+    ref, k_ref, v_ref = orc.step(case)
+    assert torch.equal(_bytes(d["k"]), _bytes(k_ref)), "K cache after the fused step"
+    assert torch.equal(_bytes(d["v"]), _bytes(v_ref)), "V cache after the fused step"
+    assert_decode_close(out, ref, case.cfg.dtype, name)
+    # the fused launch computes exactly what the two separate calls compute
+    out2, _ = gpu_step(pa, case)
+    assert torch.equal(out.cpu(), out2.cpu())
+
+
+@pytest.mark.parametrize("name", list(inputs.CONFIGS))
+def test_append_step_full_size(pa, orc, name):
+    case = inputs.make_case(name, with_post=False)
+    out, d = gpu_step_append(pa, case)
+    ref, k_ref, v_ref = orc.step(case)
+    assert torch.equal(_bytes(d["k"]), _bytes(k_ref))
+    assert torch.equal(_bytes(d["v"]), _bytes(v_ref))
+    assert_decode_close(out, ref, case.cfg.dtype, name)
+
+
+@pytest.mark.parametrize("P", [16, 64, 1024])
+def test_append_partition_sizes_and_edges(pa, orc, P):
+    case = inputs.make_case("llama3_8b_gqa", lens=[1, 15, 16, 17, 31, 32, 33, 1023, 1024, 1025, 3000])
+    out, d = gpu_step_append(pa, case, partition_size=P)
+    ref, k_ref, v_ref = orc.step(case)
+    assert torch.equal(_bytes(d["k"]), _bytes(k_ref))
+    assert_decode_close(out, ref, "bf16", f"P={P}")
