@@ -60,14 +60,18 @@ def measured_peaks():
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if any."""
+    """DRAM bytes (read + write) per decode call from the committed ncu summary,
+    or None when there is none or the kernel sources changed since it was taken."""
+    from paged_kv_cache_464_b200 import build
     path = os.path.join(ROOT, "profiles", f"pa_decode_{workload}.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return d.get("dram_bytes_per_launch")
     except Exception:
         return None
+    if d.get("source_sha256") != build.source_digest():
+        return None
+    return d.get("dram_bytes_per_call")
 
 
 # ------------------------------------------------------------------ clocks
@@ -221,13 +225,13 @@ class Step:
 def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    sampler = ClockSampler(local).start()   # started early: nvidia-smi takes a moment to report
     cfg = inputs.CONFIGS[args.workload]
     case = inputs.make_case(cfg, seed=rank_seed(cfg, rank), with_post=False)
     step = Step(case, device)
     kv_bytes = case.kv_bytes()
     stream = torch.cuda.current_stream()
 
-    sampler = ClockSampler(local).start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -275,7 +279,7 @@ def run_ours(args, world, rank, local):
     sep_ms = s_start.elapsed_time(s_stop)
 
     # keep the GPU under the same load long enough for the clock sampler
-    soak_until = wall0 + 1.5
+    soak_until = wall0 + 2.5
     while time.time() < soak_until:
         for _ in range(50):
             step()

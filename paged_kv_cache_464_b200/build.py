@@ -32,6 +32,18 @@ def sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+def source_digest() -> str:
+    """sha256 over the CUDA sources and the C header (names and contents), so a
+    recorded measurement can be matched to the kernels it was taken on."""
+    import hashlib
+    h = hashlib.sha256()
+    for path in sources():
+        h.update(os.path.basename(path).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def nvcc() -> str:
     for c in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", "nvcc"):
         if c and (os.path.isabs(c) and os.path.exists(c) or not os.path.isabs(c)):
