@@ -29,7 +29,13 @@ NVCC_FLAGS = [
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + glob.glob(os.path.join(INCLUDE, "*.h")))
+                  + glob.glob(os.path.join(CSRC, "*.cpp")) + glob.glob(os.path.join(INCLUDE, "*.h")))
+
+
+def kernel_sources():
+    """The files that define the GPU kernels and their launches."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+                  + [os.path.join(INCLUDE, "pa.h")])
 
 
 def source_digest() -> str:
@@ -37,7 +43,7 @@ def source_digest() -> str:
     recorded measurement can be matched to the kernels it was taken on."""
     import hashlib
     h = hashlib.sha256()
-    for path in sources():
+    for path in kernel_sources():
         h.update(os.path.basename(path).encode())
         with open(path, "rb") as f:
             h.update(f.read())
@@ -58,7 +64,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, "pa.cu"), "-o", LIB + ".tmp"]
+    cmd += [os.path.join(CSRC, "pa.cu"), os.path.join(CSRC, "pa_block_manager.cpp"), "-o", LIB + ".tmp"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stderr[-8000:])

@@ -10,6 +10,8 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "pa.h")
+HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+                 if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -20,10 +22,12 @@ def capi():
     return capi
 
 
-def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+def declared_functions(headers=HEADERS):
+    names = set()
+    for h in headers:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_three_calls():
@@ -38,11 +42,12 @@ def test_library_exports_every_declared_symbol(capi):
     exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
     missing = [n for n in declared_functions() if n not in exported]
     assert not missing, missing
-    assert sorted(capi.EXPORTED) == declared_functions()
+    from paged_kv_cache_464_b200 import block_manager
+    assert sorted(capi.EXPORTED + block_manager.EXPORTED) == declared_functions()
 
 
 def test_header_compiles_as_c():
-    src = f'#include "{HEADER}"\nint main(void){{ return (int)PA_OK; }}\n'
+    src = "".join(f'#include "{h}"\n' for h in HEADERS) + "int main(void){ return (int)PA_OK + (int)PA_BM_OK; }\n"
     r = subprocess.run(["gcc", "-x", "c", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-"], input=src,
                        text=True, capture_output=True)
     assert r.returncode == 0, r.stderr
