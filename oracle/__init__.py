@@ -68,6 +68,16 @@ class Oracle:
         lib.oracle_slot_for_position.argtypes = [P, I, I64, I]
         lib.oracle_widen.restype = None
         lib.oracle_widen.argtypes = [P, P, I64, I]
+        U8 = ctypes.c_void_p
+        lib.oracle_e4m3_decode.restype = None
+        lib.oracle_e4m3_decode.argtypes = [P, U8, I64]
+        lib.oracle_e4m3_quantize.restype = None
+        lib.oracle_e4m3_quantize.argtypes = [U8, P, I64, I, ctypes.c_float]
+        lib.oracle_reshape_and_cache_fp8.restype = I
+        lib.oracle_reshape_and_cache_fp8.argtypes = [U8, U8, P, P, P, I, I, I, I, I, I, ctypes.c_float,
+                                                     ctypes.c_float]
+        lib.oracle_paged_decode_fp8.restype = I
+        lib.oracle_paged_decode_fp8.argtypes = [P, P, I, U8, U8, D, D, P, I, P, I, I, I, I, I, I, D]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         self.lib = lib
@@ -146,6 +156,43 @@ class Oracle:
         if rc:
             raise OracleError(rc)
         return self.paged_decode(case.q, k, v, case.block_tables, case.context_lens, case.scale)
+
+    # -- FP8 (E4M3) caches ------------------------------------------------------------
+    def e4m3_decode(self, codes: torch.Tensor) -> np.ndarray:
+        c = codes.contiguous().view(torch.uint8)
+        out = np.empty(c.numel(), dtype=np.float64)
+        self.lib.oracle_e4m3_decode(_ptr(out), _ptr(c), c.numel())
+        return out.reshape(tuple(codes.shape))
+
+    def e4m3_quantize(self, x: torch.Tensor, scale: float) -> torch.Tensor:
+        x = x.contiguous()
+        out = torch.empty(x.shape, dtype=torch.uint8)
+        self.lib.oracle_e4m3_quantize(_ptr(out), _ptr(x), x.numel(), DTYPE_CODE[x.dtype], float(scale))
+        return out
+
+    def reshape_and_cache_fp8(self, k_cache, v_cache, key, value, slot_mapping, k_scale, v_scale):
+        """k_cache / v_cache: uint8 [NB, bs, Hkv, D], in place; returns the status code."""
+        NB, bs, Hkv, D = k_cache.shape
+        assert k_cache.dtype == torch.uint8 and k_cache.is_contiguous() and v_cache.is_contiguous()
+        sm = slot_mapping.to(torch.int64).contiguous()
+        return self.lib.oracle_reshape_and_cache_fp8(
+            _ptr(k_cache), _ptr(v_cache), _ptr(key.contiguous()), _ptr(value.contiguous()), _ptr(sm),
+            key.shape[0], Hkv, D, bs, NB, DTYPE_CODE[key.dtype], float(k_scale), float(v_scale))
+
+    def paged_decode_fp8(self, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale):
+        S, Hq, D = q.shape
+        NB, bs, Hkv, D2 = k_cache.shape
+        assert D2 == D and k_cache.dtype == torch.uint8
+        bt = block_tables.to(torch.int32).contiguous()
+        cl = context_lens.to(torch.int32).contiguous()
+        out = np.zeros((S, Hq, D), dtype=np.float64)
+        rc = self.lib.oracle_paged_decode_fp8(
+            _ptr(out), _ptr(q.contiguous()), DTYPE_CODE[q.dtype], _ptr(k_cache.contiguous()),
+            _ptr(v_cache.contiguous()), float(np.float32(k_scale)), float(np.float32(v_scale)), _ptr(bt),
+            bt.shape[1], _ptr(cl), S, Hq, Hkv, D, bs, NB, float(np.float32(scale)))
+        if rc:
+            raise OracleError(rc)
+        return out
 
     @property
     def num_threads(self) -> int:

@@ -51,6 +51,11 @@
  *                            other byte unchanged; conflict rule cases.
  *   oracle_slot_for_position the append rule against the generator's slots.
  *   oracle_widen             every fp16/bf16 bit pattern against numpy/torch.
+ *   oracle_e4m3_decode       all 256 codes against torch's float8_e4m3fn.
+ *   oracle_e4m3_quantize     torch's float8_e4m3fn cast (nearest, ties to even)
+ *                            inside the finite range; saturation outside it.
+ *   oracle_reshape_and_cache_fp8  the slot layout of oracle_reshape_and_cache.
+ *   oracle_paged_decode_fp8  torch SDPA (fp64) on the dequantised logical K/V.
  */
 #include <math.h>
 #include <stdint.h>
@@ -299,6 +304,156 @@ int oracle_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mappin
     memcpy((char *)v_cache + dst * block_bytes, (const char *)v_cache + src * block_bytes, (size_t)block_bytes);
   }
   free(ok);
+  return status;
+}
+
+/*
+ * ---------------------------------------------------------------- FP8 KV cache
+ * An 8-bit KV cache ("vLLM推理引擎深度实战：…" §四 names FP8 among vLLM's
+ * quantisation options).  Readings: the format is OCP FP8 E4M3 (sign, 4-bit
+ * exponent with bias 7, 3-bit mantissa; no infinities; codes 0x7F / 0xFF are
+ * NaN; largest finite 448); each cache has one fp32 scale; a stored code c
+ * stands for e4m3(c) * scale; a value x is stored as the E4M3 value nearest to
+ * the fp32 quotient x / scale (IEEE division), ties to the even code, values
+ * of magnitude >= 448 saturating to +-448, NaN to 0x7F.
+ */
+static double e4m3_value(uint8_t c) {
+  int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9);          /* subnormal: m * 2^-9 */
+  else
+    v = ldexp(8.0 + m, e - 10);        /* (1 + m/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* nearest E4M3 code by exhaustive search over the finite codes (ties: even code) */
+static uint8_t e4m3_encode(float x) {
+  if (isnan(x)) return 0x7F;
+  int sign = signbit(x) ? 1 : 0;
+  double a = fabs((double)x);
+  if (a >= 448.0) return (uint8_t)(sign ? 0xFE : 0x7E);
+  int best = 0;
+  double best_d = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    double d = fabs(e4m3_value((uint8_t)c) - a);
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return (uint8_t)(best | (sign << 7));
+}
+
+void oracle_e4m3_decode(double *out, const uint8_t *in, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(in[i]);
+}
+
+/* codes of widen(src[i]) / scale, src in `dtype` (f32, f16 or bf16) */
+void oracle_e4m3_quantize(uint8_t *out, const void *src, int64_t n, int dtype, float scale) {
+  for (int64_t i = 0; i < n; ++i) {
+    float x = (float)widen_one(src, i, dtype);   /* exact: every f16 / bf16 value is an f32 */
+    float q = x / scale;
+    out[i] = e4m3_encode(q);
+  }
+}
+
+/* oracle_reshape_and_cache with quantisation: rows of key / value ([T][Hkv][D]
+ * in `dtype`) are stored as E4M3 codes (k_scale, v_scale) in the 1-byte caches. */
+int oracle_reshape_and_cache_fp8(uint8_t *k_cache, uint8_t *v_cache, const void *key, const void *value,
+                                 const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                 int block_size, int num_blocks, int dtype, float k_scale, float v_scale) {
+  int status = ORACLE_OK;
+  for (int i = 0; i < num_tokens; ++i) {
+    int64_t slot = slot_mapping[i];
+    if (slot < 0) continue;
+    if (slot >= (int64_t)num_blocks * block_size) {
+      if (status == ORACLE_OK) status = ORACLE_BAD_SLOT;
+      continue;
+    }
+    int64_t block = slot / block_size;
+    int64_t offset = slot % block_size;
+    for (int h = 0; h < num_kv_heads; ++h) {
+      int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * head_dim;
+      int64_t src = ((int64_t)i * num_kv_heads + h) * head_dim;
+      for (int d = 0; d < head_dim; ++d) {
+        k_cache[dst + d] = e4m3_encode((float)widen_one(key, src + d, dtype) / k_scale);
+        v_cache[dst + d] = e4m3_encode((float)widen_one(value, src + d, dtype) / v_scale);
+      }
+    }
+  }
+  return status;
+}
+
+/*
+ * Paged decode over 1-byte E4M3 caches: exactly oracle_paged_decode with
+ * K_t[d] = e4m3(code) * k_scale and V_t[d] = e4m3(code) * v_scale (products in
+ * fp64, exact), q in `q_dtype`.
+ */
+int oracle_paged_decode_fp8(double *out, const void *q, int q_dtype, const uint8_t *k_cache,
+                            const uint8_t *v_cache, double k_scale, double v_scale,
+                            const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                            int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, double scale) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_heads % num_kv_heads != 0)
+    return ORACLE_BAD_ARGS;
+  const int group = num_heads / num_kv_heads;
+  const int64_t D = head_dim;
+  for (int b = 0; b < num_seqs; ++b) {
+    int L = context_lens[b];
+    if (L < 0 || (int64_t)L > (int64_t)max_blocks_per_seq * block_size) return ORACLE_BAD_CONTEXT_LEN;
+    for (int j = 0; j < (L + block_size - 1) / block_size; ++j) {
+      int32_t id = block_tables[(int64_t)b * max_blocks_per_seq + j];
+      if (id < 0 || id >= num_blocks) return ORACLE_BAD_BLOCK_ID;
+    }
+  }
+  int status = ORACLE_OK;
+  const int64_t rows = (int64_t)num_seqs * num_heads;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < rows; ++r) {
+    const int b = (int)(r / num_heads);
+    const int h = (int)(r % num_heads);
+    const int g = h / group;
+    const int L = context_lens[b];
+    double *o = out + r * D;
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    if (L == 0) continue;
+    double *s = (double *)malloc(sizeof(double) * (size_t)L);
+    double *qv = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!s || !qv) {
+      free(s);
+      free(qv);
+#pragma omp atomic write
+      status = ORACLE_NO_MEMORY;
+      continue;
+    }
+    for (int64_t d = 0; d < D; ++d) qv[d] = widen_one(q, r * D + d, q_dtype);
+    for (int t = 0; t < L; ++t) {
+      int32_t physical_block = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
+      int64_t row = (((int64_t)physical_block * block_size + t % block_size) * num_kv_heads + g) * D;
+      double dot = 0.0;
+      for (int64_t d = 0; d < D; ++d) dot += qv[d] * (e4m3_value(k_cache[row + d]) * k_scale);
+      s[t] = scale * dot;
+    }
+    double m = s[0];
+    for (int t = 1; t < L; ++t)
+      if (s[t] > m) m = s[t];
+    double z = 0.0;
+    for (int t = 0; t < L; ++t) {
+      s[t] = exp(s[t] - m);
+      z += s[t];
+    }
+    for (int t = 0; t < L; ++t) s[t] = s[t] / z;
+    for (int t = 0; t < L; ++t) {
+      int32_t physical_block = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
+      int64_t row = (((int64_t)physical_block * block_size + t % block_size) * num_kv_heads + g) * D;
+      for (int64_t d = 0; d < D; ++d) o[d] += s[t] * (e4m3_value(v_cache[row + d]) * v_scale);
+    }
+    free(s);
+    free(qv);
+  }
   return status;
 }
 

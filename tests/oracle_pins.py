@@ -303,6 +303,86 @@ def pin_errors(o):
         raise AssertionError("out-of-range block id not reported")
 
 
+# ---------------------------------------------------------------------------- FP8 (E4M3) cache
+def pin_e4m3_decode(o):
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    got = o.e4m3_decode(codes)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "E4M3 NaN codes"
+    assert np.array_equal(got[~nan], ref[~nan]), "E4M3 values"
+
+
+def pin_e4m3_quantize(o):
+    g = torch.Generator().manual_seed(11)
+    x = torch.cat([torch.randn(20000, generator=g) * 30,
+                   torch.randn(5000, generator=g) * 2 ** -8,                 # subnormal range
+                   (torch.arange(-256, 256, dtype=torch.float32) + 0.5) * 2 ** -9,   # exact ties
+                   torch.tensor([0.0, -0.0, 447.9, 448.0, 463.9, 464.0, -464.0, 479.9])])
+    for scale in (1.0, 0.037, 2.5):
+        got = o.e4m3_quantize(x, scale)
+        q = x / torch.tensor(scale, dtype=torch.float32)
+        inside = q.abs() <= 464          # torch's cast overflows to NaN beyond the 448/480 midpoint
+        ref = q[inside].to(torch.float8_e4m3fn).view(torch.uint8)
+        assert torch.equal(got[inside], ref), f"E4M3 rounding (scale {scale})"
+    big = torch.tensor([464.01, 480.0, 1e6, -500.0, float("inf"), float("-inf")])
+    assert o.e4m3_quantize(big, 1.0).tolist() == [0x7E, 0x7E, 0x7E, 0xFE, 0x7E, 0xFE], "saturation to +-448"
+    assert o.e4m3_quantize(torch.tensor([float("nan")]), 1.0).tolist() == [0x7F]
+
+
+def _fp8_case(name, lens, k_scale, v_scale, o):
+    """A 16-bit case whose logical K/V are written into 1-byte caches by the oracle."""
+    case = inputs.make_case(name, lens=lens, keep_logical=True)
+    NB, bs, Hkv, D = case.k_cache.shape
+    kc = torch.zeros((NB, bs, Hkv, D), dtype=torch.uint8)
+    vc = torch.zeros_like(kc)
+    rows_k, rows_v, slots = [], [], []
+    bt = case.block_tables
+    for b in range(case.cfg.num_seqs):
+        L = int(case.context_lens[b])
+        pos = torch.arange(L)
+        slots.append(bt[b, pos // bs].to(torch.int64) * bs + pos % bs)
+        rows_k.append(torch.from_numpy(case.k_logical[b]).to(case.k_cache.dtype))
+        rows_v.append(torch.from_numpy(case.v_logical[b]).to(case.k_cache.dtype))
+    sm, K, V = torch.cat(slots), torch.cat(rows_k), torch.cat(rows_v)
+    assert o.reshape_and_cache_fp8(kc, vc, K, V, sm, k_scale, v_scale) == 0
+    return case, kc, vc, K, V, sm
+
+
+def pin_fp8_cache_layout(o):
+    case, kc, vc, K, V, sm = _fp8_case("llama3_8b_gqa", [40, 17, 3], 0.02, 0.03, o)
+    NB, bs, Hkv, D = kc.shape
+    flat_k, flat_v = kc.view(NB * bs, Hkv, D), vc.view(NB * bs, Hkv, D)
+    assert torch.equal(flat_k[sm], o.e4m3_quantize(K, 0.02)), "K rows at their slots"
+    assert torch.equal(flat_v[sm], o.e4m3_quantize(V, 0.03)), "V rows at their slots"
+    untouched = torch.ones(NB * bs, dtype=torch.bool)
+    untouched[sm] = False
+    assert int(flat_k[untouched].abs().sum()) == 0 and int(flat_v[untouched].abs().sum()) == 0
+
+
+def pin_fp8_decode_vs_sdpa(o):
+    for name, lens, ks, vs in (("llama3_8b_gqa", [128, 250, 17, 5], 0.011, 0.013),
+                               ("llama2_7b", [64, 1, 77], 0.02, 0.05)):
+        case, kc, vc, K, V, sm = _fp8_case(name, lens, ks, vs, o)
+        got = o.paged_decode_fp8(case.q, kc, vc, ks, vs, case.block_tables, case.context_lens, case.scale)
+        # dense reference on the dequantised logical rows
+        dk = o.e4m3_decode(o.e4m3_quantize(K, ks)) * float(np.float32(ks))
+        dv = o.e4m3_decode(o.e4m3_quantize(V, vs)) * float(np.float32(vs))
+        c = case.cfg
+        ref = np.zeros_like(got)
+        start = 0
+        for b in range(c.num_seqs):
+            L = int(case.context_lens[b])
+            Kb = torch.from_numpy(dk[start:start + L]).permute(1, 0, 2)[None]
+            Vb = torch.from_numpy(dv[start:start + L]).permute(1, 0, 2)[None]
+            start += L
+            qb = case.q[b].to(torch.float64)[None, :, None, :]
+            ref[b] = F.scaled_dot_product_attention(qb, Kb, Vb, scale=float(np.float32(case.scale)),
+                                                    enable_gqa=True)[0, :, 0, :].numpy()
+        assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max()), f"{name}: fp8 decode vs SDPA"
+
+
 ALL_PINS = [pin_widening, pin_dense_equivalence, pin_gqa_mapping, pin_block_permutation,
             pin_length_one, pin_weights, pin_closed_forms, pin_slot_rule, pin_cache_writes,
-            pin_copy_blocks, pin_copy_on_write_invariant, pin_errors]
+            pin_copy_blocks, pin_copy_on_write_invariant, pin_errors, pin_e4m3_decode, pin_e4m3_quantize,
+            pin_fp8_cache_layout, pin_fp8_decode_vs_sdpa]

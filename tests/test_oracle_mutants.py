@@ -13,11 +13,14 @@ import oracle_pins
 
 # (name, text in pa_oracle.c, replacement).  Each must occur exactly once.
 MUTANTS = [
-    ("interleaved_gqa", "const int g = h / group;", "const int g = h % num_kv_heads;"),
-    ("dropped_scale", "s[t] = scale * dot;", "s[t] = dot;"),
-    ("sign_in_exponent", "s[t] = exp(s[t] - m);", "s[t] = exp(m - s[t]);"),
-    ("min_for_max", "if (s[t] > m) m = s[t];", "if (s[t] < m) m = s[t];"),
-    ("no_normalisation", "for (int t = 0; t < L; ++t) s[t] = s[t] / z;", "for (int t = 0; t < L; ++t) s[t] = s[t];"),
+    ("interleaved_gqa", "const int g = h / group;                       /* KV head of this query head */",
+     "const int g = h % num_kv_heads;"),
+    ("dropped_scale", "s[t] = scale * dot;\n    }\n\n    /* softmax", "s[t] = dot;\n    }\n\n    /* softmax"),
+    ("sign_in_exponent", "s[t] = exp(s[t] - m);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)",
+     "s[t] = exp(m - s[t]);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)"),
+    ("min_for_max", "if (s[t] > m) m = s[t];\n    double z = 0.0;\n    for (int t = 0; t < L; ++t) {\n      s[t] = exp(s[t] - m);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)",
+     "if (s[t] < m) m = s[t];\n    double z = 0.0;\n    for (int t = 0; t < L; ++t) {\n      s[t] = exp(s[t] - m);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)"),
+    ("no_normalisation", "for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)", "for (int t = 0; t < L; ++t) s[t] = s[t];\n    if (weights)"),
     ("value_from_key_cache", "o[d] += s[t] * widen_one(v_cache, row + d, dtype);",
      "o[d] += s[t] * widen_one(k_cache, row + d, dtype);"),
     ("kv_head_zero", "int64_t row = (((int64_t)physical_block * block_size + offset) * num_kv_heads + g) * D;\n      double dot",
@@ -36,8 +39,18 @@ MUTANTS = [
      "if ((j != i && block_mapping[2 * j + 1] == dst)) {"),
     ("copy_only_key_cache", "memcpy((char *)v_cache + dst * block_bytes, (const char *)v_cache + src * block_bytes, (size_t)block_bytes);",
      ""),
-    ("negative_slot_written", "if (slot < 0) continue;", "if (slot < 0) slot = 0;"),
-    ("weights_without_max_shift", "s[t] = exp(s[t] - m);", "s[t] = exp(s[t]);"),
+    ("negative_slot_written", "if (slot < 0) continue;\n    if (slot >= (int64_t)num_blocks * block_size) {\n      if (status == ORACLE_OK) status = ORACLE_BAD_SLOT;\n      continue;\n    }\n    int64_t block = slot / block_size;\n    int64_t offset = slot % block_size;\n    for (int h = 0; h < num_kv_heads; ++h) {\n      int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * row_bytes;",
+     "if (slot < 0) slot = 0;\n    if (slot >= (int64_t)num_blocks * block_size) {\n      if (status == ORACLE_OK) status = ORACLE_BAD_SLOT;\n      continue;\n    }\n    int64_t block = slot / block_size;\n    int64_t offset = slot % block_size;\n    for (int h = 0; h < num_kv_heads; ++h) {\n      int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * row_bytes;"),
+    ("weights_without_max_shift", "s[t] = exp(s[t] - m);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)",
+     "s[t] = exp(s[t]);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)"),
+    ("e4m3_bias", "v = ldexp(8.0 + m, e - 10);", "v = ldexp(8.0 + m, e - 9);"),
+    ("e4m3_ties_to_odd", "(d == best_d && (c & 1) == 0)", "(d == best_d && (c & 1) == 1)"),
+    ("e4m3_no_saturation", "if (a >= 448.0) return (uint8_t)(sign ? 0xFE : 0x7E);", "if (a >= 1e30) return 0;"),
+    ("e4m3_multiply_by_scale", "float q = x / scale;", "float q = x * scale;"),
+    ("fp8_v_scale_dropped", "o[d] += s[t] * (e4m3_value(v_cache[row + d]) * v_scale);",
+     "o[d] += s[t] * e4m3_value(v_cache[row + d]);"),
+    ("fp8_write_k_with_v_scale", "k_cache[dst + d] = e4m3_encode((float)widen_one(key, src + d, dtype) / k_scale);",
+     "k_cache[dst + d] = e4m3_encode((float)widen_one(key, src + d, dtype) / v_scale);"),
 ]
 
 
