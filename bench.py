@@ -193,19 +193,40 @@ class Step:
         ws = capi.decode_workspace_bytes(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, self.maxL, self.P)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
         self.has_pairs = case.block_mapping.numel() > 0
+        self.fp8 = c.kv_dtype == "fp8_e4m3"
+        if self.fp8:
+            # 1-byte caches: quantise the whole pool once (setup, not timed)
+            nb, bs, hkv, d = self.k.shape
+            self.kv_scale = c.kv_scale
+            k8 = torch.zeros((nb, bs, hkv, d), dtype=torch.uint8, device=device)
+            v8 = torch.zeros_like(k8)
+            slots = torch.arange(nb * bs, dtype=torch.int64, device=device)
+            capi.reshape_and_cache_fp8(self.k.view(nb * bs, hkv, d), self.v.view(nb * bs, hkv, d), k8, v8, slots,
+                                       self.kv_scale, self.kv_scale)
+            torch.cuda.synchronize()
+            self.k, self.v = k8, v8
 
     def launches(self, fused: bool) -> int:
         c = self.case.cfg
         P = self.pa.decode_partition_size(c.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, self.maxL, self.P)
         split = math.ceil(self.maxL / P) > 1
-        return (1 if self.has_pairs else 0) + (0 if fused else 1) + 1 + (1 if split else 0)
+        return (1 if self.has_pairs else 0) + (0 if fused and not self.fp8 else 1) + 1 + (1 if split else 0)
 
-    # fused step: copies, then the new-token write and decode in one launch (pa_decode_append)
+    # fused step: copies, then the new-token write and decode in one launch (pa_decode_append);
+    # 1-byte caches: copies, the quantising new-token write, then pa_decode_fp8
     def pre(self):
         if self.has_pairs:
             self.pa.copy_blocks(self.k, self.v, self.pairs)
+        if self.fp8:
+            self.pa.reshape_and_cache_fp8(self.key, self.value, self.k, self.v, self.slots, self.kv_scale,
+                                          self.kv_scale)
 
     def decode(self):
+        if self.fp8:
+            self.pa.decode_fp8(self.q, self.k, self.v, self.kv_scale, self.kv_scale, self.bt, self.cl,
+                               self.case.scale, out=self.out, max_context_len=self.maxL, partition_size=self.P,
+                               workspace=self.ws)
+            return
         self.pa.decode_append(self.q, self.key, self.value, self.k, self.v, self.bt, self.cl, self.case.scale,
                               out=self.out, max_context_len=self.maxL, partition_size=self.P, workspace=self.ws)
 
@@ -215,6 +236,9 @@ class Step:
 
     # the same step as three separate calls (pa_copy_blocks, pa_reshape_and_cache, pa_decode)
     def separate(self):
+        if self.fp8:
+            self()
+            return
         if self.has_pairs:
             self.pa.copy_blocks(self.k, self.v, self.pairs)
         self.pa.reshape_and_cache(self.key, self.value, self.k, self.v, self.slots)
@@ -316,7 +340,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": cfg.dtype,
+        "dtype": "fp8_e4m3 KV (f16 tensor-core math), bf16 q/out" if step.fp8 else cfg.dtype,
         "data": "synthetic (seeded N(0,1) Q/K/V, shuffled block pool)",
         "config": {
             "workload": cfg.name,
@@ -330,18 +354,22 @@ def run_ours(args, world, rank, local):
             "kv_bytes_per_step_per_gpu": kv_bytes,
             "partition_size": step.pa.decode_partition_size(cfg.num_seqs, cfg.num_heads, cfg.num_kv_heads,
                                                             cfg.head_dim, step.maxL, step.P),
-            "step": ("pa_copy_blocks + " if step.has_pairs else "") + "pa_decode_append (new-token write + decode)",
+            "step": ("pa_copy_blocks + " if step.has_pairs else "") + (
+                "pa_reshape_and_cache_fp8 + pa_decode_fp8" if step.fp8 else
+                "pa_decode_append (new-token write + decode)"),
+            "kv_cache": "fp8_e4m3, scale %g" % cfg.kv_scale if step.fp8 else cfg.dtype,
             "l2": f"inputs larger than L2: {kv_bytes / 2**20:.0f} MiB of KV per step vs 126 MiB L2, no flush",
             "parallelism": f"replicas x{world}, no data-path collective",
         },
         "seqs_per_s": round(total_seqs * args.steps / (max_ms * 1e-3), 1),
         "step_separate_calls": {
-            "calls": ("pa_copy_blocks + " if step.has_pairs else "") + "pa_reshape_and_cache + pa_decode",
+            "calls": ("pa_copy_blocks + " if step.has_pairs else "") + (
+                "pa_reshape_and_cache_fp8 + pa_decode_fp8" if step.fp8 else "pa_reshape_and_cache + pa_decode"),
             "value": round(total_bytes * args.steps / (sep_max_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(sep_max_ms / args.steps, 5)},
         "pct_hbm_peak": round(100.0 * value / world / peak, 2),
         "roofline": {
-            "kernel": "pa_decode_append (partition + reduce launches)",
+            "kernel": ("pa_decode_fp8" if step.fp8 else "pa_decode_append") + " (partition + reduce launches)",
             "bound": "hbm",
             "achieved": round(achieved, 2),
             "peak": peak,
@@ -415,16 +443,39 @@ def _sample_case(case: inputs.DecodeCase, n: int) -> inputs.DecodeCase:
                                context_lens=case.context_lens[:n])
 
 
+def _oracle_caches(o, case):
+    """The oracle's own copy of the pre-step caches (1-byte codes for FP8 workloads)."""
+    if case.cfg.kv_dtype != "fp8_e4m3":
+        return case.k_cache.clone(), case.v_cache.clone()
+    nb, bs, hkv, d = case.k_cache.shape
+    k8 = torch.zeros((nb, bs, hkv, d), dtype=torch.uint8)
+    v8 = torch.zeros_like(k8)
+    slots = torch.arange(nb * bs, dtype=torch.int64)
+    o.reshape_and_cache_fp8(k8, v8, case.k_cache.view(nb * bs, hkv, d), case.v_cache.view(nb * bs, hkv, d), slots,
+                            case.cfg.kv_scale, case.cfg.kv_scale)
+    return k8, v8
+
+
+def _oracle_step(o, case, k, v):
+    if case.cfg.kv_dtype != "fp8_e4m3":
+        return o.step_inplace(case, k, v)
+    s = case.cfg.kv_scale
+    if case.block_mapping.numel():
+        o.copy_blocks(k.view(torch.bfloat16), v.view(torch.bfloat16), case.block_mapping)
+    o.reshape_and_cache_fp8(k, v, case.key, case.value, case.slot_mapping, s, s)
+    return o.paged_decode_fp8(case.q, k, v, s, s, case.block_tables, case.context_lens, case.scale)
+
+
 def cpu_baseline(case, budget_s: float = 20.0):
     """The oracle, as it stands, on the host cores: one step on a bounded sample.
     The caches are cloned once outside the timed region (the step is idempotent)."""
     import oracle
     o = oracle.get()
-    k, v = case.k_cache.clone(), case.v_cache.clone()
+    k, v = _oracle_caches(o, case)
     # calibrate on a few sequences, then size the sample to the budget
     n0 = min(4, case.cfg.num_seqs)
     t = time.perf_counter()
-    o.step_inplace(_sample_case(case, n0), k, v)
+    _oracle_step(o, _sample_case(case, n0), k, v)
     per_seq = (time.perf_counter() - t) / n0
     n = max(1, min(case.cfg.num_seqs, int(budget_s / 2 / max(per_seq, 1e-6))))
     sample = _sample_case(case, n)
@@ -433,7 +484,7 @@ def cpu_baseline(case, budget_s: float = 20.0):
     t_all = time.perf_counter()
     while reps < 3 and (reps == 0 or time.perf_counter() - t_all < budget_s / 2):
         t = time.perf_counter()
-        o.step_inplace(sample, k, v)
+        _oracle_step(o, sample, k, v)
         dt = time.perf_counter() - t
         best = dt if best is None else min(best, dt)
         reps += 1
@@ -451,20 +502,20 @@ def run_reference(args, world, rank):
     o = oracle.get()
     cfg = inputs.CONFIGS[args.workload]
     case = inputs.make_case(cfg, seed=rank_seed(cfg, 0), with_post=False)
-    k, v = case.k_cache.clone(), case.v_cache.clone()
+    k, v = _oracle_caches(o, case)
     # size each step so that warm-up + timed steps take about `ref_budget` seconds
     n0 = min(4, cfg.num_seqs)
     t = time.perf_counter()
-    o.step_inplace(_sample_case(case, n0), k, v)
+    _oracle_step(o, _sample_case(case, n0), k, v)
     per_seq = (time.perf_counter() - t) / n0
     per_step_budget = args.ref_budget / max(1, args.steps + args.warmup)
     n = max(1, min(cfg.num_seqs, int(per_step_budget / max(per_seq, 1e-6))))
     sample = _sample_case(case, n)
     for _ in range(args.warmup):
-        o.step_inplace(sample, k, v)
+        _oracle_step(o, sample, k, v)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        o.step_inplace(sample, k, v)
+        _oracle_step(o, sample, k, v)
     el = time.perf_counter() - t0
     value = sample.kv_bytes() * args.steps / el / 1e9
     desc = (f"first {n} of {cfg.num_seqs} sequences per step (copies, new-token write, fp64 decode), "

@@ -32,7 +32,8 @@
  *   [num_blocks][block_size][num_kv_heads][head_dim], row-major, contiguous
  *   (token-major inside a block, the per-block layout of [A] §五 with the K/V
  *   axis split into two tensors).  block_size must be 16.  One (token, KV head)
- *   row must be 256 bytes: head_dim 64 for PA_F32, 128 for PA_F16 / PA_BF16.
+ *   row must be 256 bytes: head_dim 64 for PA_F32, 128 for PA_F16 / PA_BF16 --
+ *   or 128 bytes for 1-byte PA_FP8_E4M3 caches (head_dim 128).
  *   Cache base addresses must be 16-byte aligned.
  * - A slot is a flat token index into the pool: slot = physical_block *
  *   block_size + offset ([A] §三 append_token: a new token goes to the next
@@ -48,7 +49,9 @@
 extern "C" {
 #endif
 
-typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype_t;
+/* PA_FP8_E4M3: 1-byte OCP E4M3 codes with one fp32 scale per cache (see
+ * pa_reshape_and_cache_fp8); only for caches. */
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_FP8_E4M3 = 3 } pa_dtype_t;
 
 typedef enum {
   PA_OK = 0,
@@ -90,6 +93,25 @@ pa_status_t pa_reshape_and_cache(const void *key, const void *value, void *k_cac
                                  const int64_t *slot_mapping, int num_tokens, int64_t num_blocks,
                                  int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype,
                                  void *stream);
+
+/*
+ * pa_reshape_and_cache_fp8 -- pa_reshape_and_cache into 1-byte E4M3 caches.
+ * (An 8-bit KV cache: "vLLM推理引擎深度实战：…" §四 lists FP8 among vLLM's
+ * quantisation options.)
+ *
+ * key, value    [num_tokens][num_kv_heads][128] in src_dtype (PA_F16 or PA_BF16).
+ * k_cache, v_cache  [num_blocks][16][num_kv_heads][128] bytes.
+ * Element x of a key row is stored as the OCP E4M3 code nearest to the fp32
+ * quotient x / k_scale (IEEE division), ties to even, saturating at +-448
+ * (NaN gives a NaN code); likewise value with v_scale.  Scales are finite and
+ * > 0.  Slots as in pa_reshape_and_cache.
+ * Errors: as pa_reshape_and_cache; PA_ERR_DTYPE for another src_dtype,
+ * PA_ERR_SHAPE for head_dim != 128 or a bad scale.
+ */
+pa_status_t pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
+                                     const int64_t *slot_mapping, int num_tokens, int64_t num_blocks,
+                                     int block_size, int num_kv_heads, int head_dim, pa_dtype_t src_dtype,
+                                     float k_scale, float v_scale, void *stream);
 
 /*
  * pa_decode_partition_size -- the partition size (tokens per split-K piece)
@@ -146,6 +168,23 @@ pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void 
                       int max_context_len, float scale, int partition_size, void *workspace,
                       size_t workspace_bytes, int64_t num_blocks, int block_size, int num_kv_heads,
                       int head_dim, pa_dtype_t dtype, void *stream);
+
+/*
+ * pa_decode_fp8 -- pa_decode over 1-byte E4M3 caches (head_dim 128).
+ *
+ * K_t[d] = e4m3(k_cache code) * k_scale and V_t[d] = e4m3(v_cache code) *
+ * v_scale; q and out are in q_dtype (PA_F16 or PA_BF16).  The tensor cores
+ * compute in fp16 with fp32 accumulation: q is converted to fp16 once (exact
+ * inside the fp16 normal range, |q| in [6.1e-5, 65504]); E4M3 codes convert to
+ * fp16 exactly.  Everything else -- arguments, workspace, errors, group sizes
+ * 1..8 -- as pa_decode.
+ */
+pa_status_t pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache, float k_scale,
+                          float v_scale, const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len,
+                          float scale, int partition_size, void *workspace, size_t workspace_bytes,
+                          int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                          pa_dtype_t q_dtype, void *stream);
 
 /*
  * pa_decode_append -- the decode step's new-token write and decode in one

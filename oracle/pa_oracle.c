@@ -328,6 +328,12 @@ static double e4m3_value(uint8_t c) {
   return sign ? -v : v;
 }
 
+/* the values of the non-negative finite codes 0x00..0x7E (filled before use) */
+static double e4m3_positive[0x7F];
+static void e4m3_fill_table(void) {
+  for (int c = 0; c <= 0x7E; ++c) e4m3_positive[c] = e4m3_value((uint8_t)c);
+}
+
 /* nearest E4M3 code by exhaustive search over the finite codes (ties: even code) */
 static uint8_t e4m3_encode(float x) {
   if (isnan(x)) return 0x7F;
@@ -337,7 +343,7 @@ static uint8_t e4m3_encode(float x) {
   int best = 0;
   double best_d = INFINITY;
   for (int c = 0; c <= 0x7E; ++c) {
-    double d = fabs(e4m3_value((uint8_t)c) - a);
+    double d = fabs(e4m3_positive[c] - a);
     if (d < best_d || (d == best_d && (c & 1) == 0)) {
       best = c;
       best_d = d;
@@ -352,6 +358,8 @@ void oracle_e4m3_decode(double *out, const uint8_t *in, int64_t n) {
 
 /* codes of widen(src[i]) / scale, src in `dtype` (f32, f16 or bf16) */
 void oracle_e4m3_quantize(uint8_t *out, const void *src, int64_t n, int dtype, float scale) {
+  e4m3_fill_table();
+#pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < n; ++i) {
     float x = (float)widen_one(src, i, dtype);   /* exact: every f16 / bf16 value is an f32 */
     float q = x / scale;
@@ -365,13 +373,13 @@ int oracle_reshape_and_cache_fp8(uint8_t *k_cache, uint8_t *v_cache, const void 
                                  const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
                                  int block_size, int num_blocks, int dtype, float k_scale, float v_scale) {
   int status = ORACLE_OK;
+  e4m3_fill_table();
+  for (int i = 0; i < num_tokens; ++i)
+    if (slot_mapping[i] >= (int64_t)num_blocks * block_size) status = ORACLE_BAD_SLOT;
+#pragma omp parallel for schedule(static)
   for (int i = 0; i < num_tokens; ++i) {
     int64_t slot = slot_mapping[i];
-    if (slot < 0) continue;
-    if (slot >= (int64_t)num_blocks * block_size) {
-      if (status == ORACLE_OK) status = ORACLE_BAD_SLOT;
-      continue;
-    }
+    if (slot < 0 || slot >= (int64_t)num_blocks * block_size) continue;
     int64_t block = slot / block_size;
     int64_t offset = slot % block_size;
     for (int h = 0; h < num_kv_heads; ++h) {

@@ -34,6 +34,11 @@ _lib.pa_decode_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I
 _lib.pa_decode_static_workspace.restype = _I
 _lib.pa_decode_static_workspace.argtypes = [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _F, _I, _I64, _I, _I, _I, _I,
                                             _P]
+_lib.pa_reshape_and_cache_fp8.restype = _I
+_lib.pa_reshape_and_cache_fp8.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _F, _F, _P]
+_lib.pa_decode_fp8.restype = _I
+_lib.pa_decode_fp8.argtypes = [_P, _P, _P, _P, _F, _F, _P, _I, _P, _I, _I, _I, _F, _I, _P, _SZ, _I64, _I, _I, _I, _I,
+                               _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I64, _I, _I, _I, _I, _P]
 _lib.pa_get_device_error.restype = _I
@@ -42,10 +47,12 @@ _lib.pa_status_string.restype = ctypes.c_char_p
 _lib.pa_status_string.argtypes = [_I]
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_append", "pa_decode_static_workspace", "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
+            "pa_decode_append", "pa_decode_static_workspace", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
 STATIC_WORKSPACE_BYTES = 64 << 20   # PA_STATIC_WORKSPACE_BYTES in include/pa.h
 
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+FP8 = 3                      # PA_FP8_E4M3: 1-byte caches held as torch.uint8 or torch.float8_e4m3fn
+FP8_TORCH = (torch.uint8, torch.float8_e4m3fn)
 DEVICE_ERRORS = {0: "ok", 1: "block id out of range", 2: "slot out of range", 3: "copy pair conflict",
                  4: "bad context length", 5: "wait timeout"}
 
@@ -81,10 +88,10 @@ def _dev(t: torch.Tensor, name: str) -> int:
 def _cache_args(k_cache: torch.Tensor, v_cache: torch.Tensor):
     if k_cache.dim() != 4 or k_cache.shape != v_cache.shape or k_cache.dtype != v_cache.dtype:
         raise ValueError("k_cache and v_cache must both be [num_blocks, block_size, num_kv_heads, head_dim]")
-    if k_cache.dtype not in DTYPE_CODE:
+    if k_cache.dtype not in DTYPE_CODE and k_cache.dtype not in FP8_TORCH:
         raise ValueError(f"unsupported cache dtype {k_cache.dtype}")
     nb, bs, hkv, d = k_cache.shape
-    return nb, bs, hkv, d, DTYPE_CODE[k_cache.dtype]
+    return nb, bs, hkv, d, (FP8 if k_cache.dtype in FP8_TORCH else DTYPE_CODE[k_cache.dtype])
 
 
 def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -214,6 +221,58 @@ def decode_static_workspace(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"), S, hq,
         max_context_len, float(scale), partition_size, nb, bs, hkv, d, dt, _stream(stream)),
         "pa_decode_static_workspace")
+    return out
+
+
+def reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                          slot_mapping: torch.Tensor, k_scale: float, v_scale: float,
+                          stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Quantise key/value rows [T, Hkv, 128] (fp16/bf16) into 1-byte E4M3 caches at their slots."""
+    nb, bs, hkv, d, dt = _cache_args(k_cache, v_cache)
+    if dt != FP8 or key.dtype not in (torch.float16, torch.bfloat16) or value.dtype != key.dtype:
+        raise ValueError("1-byte caches and fp16/bf16 key/value expected")
+    T = key.shape[0]
+    if tuple(key.shape) != (T, hkv, d) or tuple(value.shape) != (T, hkv, d) or slot_mapping.numel() != T:
+        raise ValueError("key/value must be [T, num_kv_heads, head_dim] with T slots")
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    _check(_lib.pa_reshape_and_cache_fp8(_dev(key, "key"), _dev(value, "value"), _dev(k_cache, "k_cache"),
+                                         _dev(v_cache, "v_cache"),
+                                         _dev(slot_mapping, "slot_mapping") if T else None, T, nb, bs, hkv, d,
+                                         DTYPE_CODE[key.dtype], float(k_scale), float(v_scale), _stream(stream)),
+           "pa_reshape_and_cache_fp8")
+
+
+def decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale: float, v_scale: float,
+               block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+               out: Optional[torch.Tensor] = None, *, max_context_len: Optional[int] = None,
+               partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Paged decode over 1-byte E4M3 caches; q/out fp16 or bf16."""
+    nb, bs, hkv, d, dt = _cache_args(k_cache, v_cache)
+    S, hq, dq = q.shape
+    if dt != FP8 or q.dtype not in (torch.float16, torch.bfloat16) or dq != d:
+        raise ValueError("1-byte caches and fp16/bf16 q [S, Hq, head_dim] expected")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("block_tables must be [S, max_blocks_per_seq] and context_lens [S]")
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if S else 0
+    need = decode_workspace_bytes(S, hq, hkv, d, max_context_len, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.pa_decode_fp8(_dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                              float(k_scale), float(v_scale), _dev(block_tables, "block_tables"),
+                              block_tables.shape[1], _dev(context_lens, "context_lens"), S, hq, max_context_len,
+                              float(scale), partition_size, ws_ptr, ws_bytes, nb, bs, hkv, d, DTYPE_CODE[q.dtype],
+                              _stream(stream)), "pa_decode_fp8")
     return out
 
 

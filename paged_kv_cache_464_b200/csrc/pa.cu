@@ -32,16 +32,20 @@ int elem_bytes(pa_dtype_t dt) {
     case PA_F32: return 4;
     case PA_F16:
     case PA_BF16: return 2;
+    case PA_FP8_E4M3: return 1;
   }
   return 0;
 }
+
+// Bytes of one (token, KV head) row: 256 for 16/32-bit caches, 128 for E4M3.
+int row_bytes(pa_dtype_t dt) { return dt == PA_FP8_E4M3 ? 128 : kRowBytes; }
 
 pa_status_t cache_shape_status(int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
                                pa_dtype_t dtype) {
   const int es = elem_bytes(dtype);
   if (es == 0) return PA_ERR_DTYPE;
   if (num_blocks <= 0 || num_blocks > INT32_MAX || block_size != kBlockSize || num_kv_heads <= 0 ||
-      head_dim * es != kRowBytes)
+      head_dim * es != row_bytes(dtype))
     return PA_ERR_SHAPE;
   return PA_OK;
 }
@@ -82,17 +86,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// The cache [NB][16][Hkv][256 B] seen as a 5-D byte tensor
-// {128 B, 2 halves, Hkv, 16 tokens, NB}; the box is one half of one
+// The cache [NB][16][Hkv][R B] (R = 256 or 128) seen as a 5-D byte tensor
+// {128 B, R/128 parts, Hkv, 16 tokens, NB}; the box is one 128-byte part of one
 // (block, KV head) tile: {128, 1, 1, 16, 1} = 2 KiB (16 rows of 128 B),
-// landing 128-byte swizzled.  Two boxes make the 4 KiB tile.
-bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int num_kv_heads) {
+// landing 128-byte swizzled.  R/128 boxes make the tile.
+bool encode_cache_map(CUtensorMap *map, const void *cache, int64_t num_blocks, int num_kv_heads, int rb) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[5] = {128, kRowBytes / 128, (cuuint64_t)num_kv_heads, (cuuint64_t)kBlockSize,
+  const cuuint64_t dims[5] = {128, (cuuint64_t)rb / 128, (cuuint64_t)num_kv_heads, (cuuint64_t)kBlockSize,
                               (cuuint64_t)num_blocks};
-  const cuuint64_t strides[4] = {128, (cuuint64_t)kRowBytes, (cuuint64_t)num_kv_heads * kRowBytes,
-                                 (cuuint64_t)kBlockSize * num_kv_heads * kRowBytes};
+  const cuuint64_t strides[4] = {128, (cuuint64_t)rb, (cuuint64_t)num_kv_heads * rb,
+                                 (cuuint64_t)kBlockSize * num_kv_heads * rb};
   const cuuint32_t box[5] = {128, 1, 1, kBlockSize, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void *>(cache), dims, strides, box,
@@ -181,6 +185,19 @@ pa_status_t dispatch_group(int group, const CUtensorMap &mk, const CUtensorMap &
   return PA_ERR_SHAPE;
 }
 
+// 1-byte E4M3 caches: tensor-core block math in fp16 for every group size
+template <typename T>
+pa_status_t dispatch_group_fp8(int group, const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
+                               cudaStream_t s) {
+  switch (group) {
+    case 1: return launch_decode<T, 1, pa::Fp8MmaMath<T, 1>>(mk, mv, p, s);
+    case 2: return launch_decode<T, 2, pa::Fp8MmaMath<T, 2>>(mk, mv, p, s);
+    case 4: return launch_decode<T, 4, pa::Fp8MmaMath<T, 4>>(mk, mv, p, s);
+    case 8: return launch_decode<T, 8, pa::Fp8MmaMath<T, 8>>(mk, mv, p, s);
+  }
+  return PA_ERR_SHAPE;
+}
+
 }  // namespace
 
 extern "C" {
@@ -197,7 +214,7 @@ pa_status_t pa_reshape_and_cache(const void *key, const void *value, void *k_cac
   if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
       !aligned(slot_mapping, 8))
     return PA_ERR_ALIGN;
-  const int chunks_per_slot = num_kv_heads * (kRowBytes / 16);
+  const int chunks_per_slot = num_kv_heads * (row_bytes(dtype) / 16);
   const long long total = (long long)num_tokens * chunks_per_slot;
   long long blocks = (total + 255) / 256;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
@@ -224,13 +241,17 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, 
 
 namespace {
 
+// dtype: the cache dtype; q_dtype: q and out (equal to dtype except for E4M3 caches)
 pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void *new_v, const void *k_cache,
                         const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                         const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len, float scale,
                         int partition_size, void *workspace, size_t workspace_bytes, int64_t num_blocks,
-                        int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream) {
+                        int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream,
+                        pa_dtype_t q_dtype, float k_scale, float v_scale) {
   pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
   if (st != PA_OK) return st;
+  if (dtype == PA_FP8_E4M3 ? (q_dtype != PA_F16 && q_dtype != PA_BF16) : q_dtype != dtype) return PA_ERR_DTYPE;
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f) return PA_ERR_SHAPE;
   if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 || max_blocks_per_seq < 0 ||
       num_heads % num_kv_heads != 0 || !std::isfinite(scale))
     return PA_ERR_SHAPE;
@@ -254,8 +275,8 @@ pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void 
   }
 
   CUtensorMap mk, mv;
-  if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads) ||
-      !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads))
+  if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, row_bytes(dtype)) ||
+      !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, row_bytes(dtype)))
     return PA_ERR_CUDA;
 
   pa::DecodeParams p{};
@@ -275,17 +296,22 @@ pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void 
   p.max_context_len = max_context_len;
   p.partition_size = P;
   p.max_partitions = np;
-  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (double)k_scale);
+  p.v_scale = v_scale;
   p.new_k = new_k;
   p.new_v = new_v;
   p.k_cache = new_k ? const_cast<void *>(k_cache) : nullptr;
   p.v_cache = new_k ? const_cast<void *>(v_cache) : nullptr;
 
   cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == PA_FP8_E4M3)
+    return q_dtype == PA_F16 ? dispatch_group_fp8<__half>(group, mk, mv, p, s)
+                             : dispatch_group_fp8<__nv_bfloat16>(group, mk, mv, p, s);
   switch (dtype) {
     case PA_F32: return dispatch_group<float>(group, mk, mv, p, s);
     case PA_F16: return dispatch_group<__half>(group, mk, mv, p, s);
     case PA_BF16: return dispatch_group<__nv_bfloat16>(group, mk, mv, p, s);
+    case PA_FP8_E4M3: break;
   }
   return PA_ERR_DTYPE;
 }
@@ -299,9 +325,49 @@ pa_status_t pa_decode(void *out, const void *q, const void *k_cache, const void 
                       int num_seqs, int num_heads, int max_context_len, float scale, int partition_size,
                       void *workspace, size_t workspace_bytes, int64_t num_blocks, int block_size,
                       int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream) {
+  if (dtype == PA_FP8_E4M3) return PA_ERR_DTYPE;   // pa_decode_fp8
   return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                      num_seqs, num_heads, max_context_len, scale, partition_size, workspace, workspace_bytes,
-                     num_blocks, block_size, num_kv_heads, head_dim, dtype, stream);
+                     num_blocks, block_size, num_kv_heads, head_dim, dtype, stream, dtype, 1.f, 1.f);
+}
+
+pa_status_t pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache, float k_scale,
+                          float v_scale, const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len,
+                          float scale, int partition_size, void *workspace, size_t workspace_bytes,
+                          int64_t num_blocks, int block_size, int num_kv_heads, int head_dim, pa_dtype_t q_dtype,
+                          void *stream) {
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     num_seqs, num_heads, max_context_len, scale, partition_size, workspace, workspace_bytes,
+                     num_blocks, block_size, num_kv_heads, head_dim, PA_FP8_E4M3, stream, q_dtype, k_scale, v_scale);
+}
+
+pa_status_t pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
+                                     const int64_t *slot_mapping, int num_tokens, int64_t num_blocks,
+                                     int block_size, int num_kv_heads, int head_dim, pa_dtype_t src_dtype,
+                                     float k_scale, float v_scale, void *stream) {
+  pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, PA_FP8_E4M3);
+  if (st != PA_OK) return st;
+  if (src_dtype != PA_F16 && src_dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || k_scale <= 0.f || v_scale <= 0.f) return PA_ERR_SHAPE;
+  if (num_tokens < 0) return PA_ERR_SHAPE;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_NULL;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_ALIGN;
+  const int chunks_per_slot = num_kv_heads * (head_dim / 8);   // 8 elements per thread
+  const long long total = (long long)num_tokens * chunks_per_slot;
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  const long long slots = (long long)num_blocks * block_size;
+  if (src_dtype == PA_F16)
+    return launch(pa::reshape_and_cache_fp8_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0,
+                  (cudaStream_t)stream, (const uint4 *)key, (const uint4 *)value, (uint2 *)k_cache,
+                  (uint2 *)v_cache, slot_mapping, num_tokens, chunks_per_slot, slots, k_scale, v_scale);
+  return launch(pa::reshape_and_cache_fp8_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0,
+                (cudaStream_t)stream, (const uint4 *)key, (const uint4 *)value, (uint2 *)k_cache, (uint2 *)v_cache,
+                slot_mapping, num_tokens, chunks_per_slot, slots, k_scale, v_scale);
 }
 
 pa_status_t pa_decode_append(void *out, const void *q, const void *key, const void *value, void *k_cache,
@@ -312,9 +378,10 @@ pa_status_t pa_decode_append(void *out, const void *q, const void *key, const vo
                              void *stream) {
   if (num_seqs > 0 && (!key || !value)) return PA_ERR_NULL;
   if (!aligned(key, 16) || !aligned(value, 16)) return PA_ERR_ALIGN;
+  if (dtype == PA_FP8_E4M3) return PA_ERR_DTYPE;
   return decode_impl(out, q, key, value, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                      num_seqs, num_heads, max_context_len, scale, partition_size, workspace, workspace_bytes,
-                     num_blocks, block_size, num_kv_heads, head_dim, dtype, stream);
+                     num_blocks, block_size, num_kv_heads, head_dim, dtype, stream, dtype, 1.f, 1.f);
 }
 
 pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
@@ -326,7 +393,7 @@ pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_ma
   if (num_pairs == 0) return PA_OK;
   if (!k_cache || !v_cache || !block_mapping) return PA_ERR_NULL;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8)) return PA_ERR_ALIGN;
-  const int chunks_per_block = kBlockSize * num_kv_heads * (kRowBytes / 16);
+  const int chunks_per_block = kBlockSize * num_kv_heads * (row_bytes(dtype) / 16);
   return launch(pa::copy_blocks_kernel, dim3((unsigned)num_pairs, 2), dim3(256), 0, (cudaStream_t)stream,
                 (uint4 *)k_cache, (uint4 *)v_cache, (const long long *)block_mapping, num_pairs,
                 (long long)num_blocks, chunks_per_block);

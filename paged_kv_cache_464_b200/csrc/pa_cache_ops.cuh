@@ -40,6 +40,53 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4 *__r
   }
 }
 
+// Slot write into 1-byte E4M3 caches: each stored code is the E4M3 value
+// nearest to the fp32 quotient x / scale (IEEE division), ties to even,
+// saturating at +-448 (cvt.rn.satfinite).  One thread converts 8 elements (one
+// 16-byte chunk of a 16-bit source row) into 8 codes.
+template <typename T>
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4 *__restrict__ key,
+                                                                    const uint4 *__restrict__ value,
+                                                                    uint2 *__restrict__ k_cache,
+                                                                    uint2 *__restrict__ v_cache,
+                                                                    const int64_t *__restrict__ slot_mapping,
+                                                                    int num_tokens, int chunks_per_slot,
+                                                                    long long num_slots, float k_scale,
+                                                                    float v_scale) {
+  pdl_wait();
+  pdl_trigger();
+  const long long total = static_cast<long long>(num_tokens) * chunks_per_slot;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int tok = static_cast<int>(i / chunks_per_slot);
+    const int rem = static_cast<int>(i - static_cast<long long>(tok) * chunks_per_slot);
+    const uint4 kx = key[i];
+    const uint4 vx = value[i];
+    const long long slot = slot_mapping[tok];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (rem == 0) record_error(2 /*PA_DEV_BAD_SLOT*/, slot);
+      continue;
+    }
+    float kf[8], vf[8];
+    Elem<T>::unpack(kx, kf);
+    Elem<T>::unpack(vx, vf);
+    uint32_t kc[4], vc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint16_t a, b;
+      // cvt packs its first source into the upper byte: element 2j goes low
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(a) : "f"(kf[2 * j + 1] / k_scale), "f"(kf[2 * j] / k_scale));
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(b) : "f"(vf[2 * j + 1] / v_scale), "f"(vf[2 * j] / v_scale));
+      kc[j] = a;
+      vc[j] = b;
+    }
+    const long long dst = slot * chunks_per_slot + rem;
+    k_cache[dst] = make_uint2(kc[0] | (kc[1] << 16), kc[2] | (kc[3] << 16));
+    v_cache[dst] = make_uint2(vc[0] | (vc[1] << 16), vc[2] | (vc[3] << 16));
+  }
+}
+
 // Copy-on-write block copy ("vLLM 原理与源码阅读", Block 管理器, item 3).
 // blockIdx.x = pair, blockIdx.y = 0 for the K cache, 1 for the V cache.
 // Every CTA first checks its pair against all pairs (conflicting pairs are

@@ -66,8 +66,7 @@ namespace pa {
 #endif
 constexpr int kDecodeWarps = PA_DECODE_WARPS;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
-constexpr int kStagesPerWarp = PA_DECODE_STAGES_PER_WARP;
-constexpr int kStages = kDecodeWarps * kStagesPerWarp;
+constexpr int kStagesPerWarp = PA_DECODE_STAGES_PER_WARP;   // for 256-byte rows; 128-byte rows take twice as many
 
 struct DecodeParams {
   void *out;                      // [S][Hq][D]
@@ -80,7 +79,8 @@ struct DecodeParams {
   long long num_blocks;
   int num_seqs, num_heads, num_kv_heads, max_blocks_per_seq;
   int max_context_len, partition_size, max_partitions;
-  float scale_log2;               // scale * log2(e)
+  float scale_log2;               // scale * log2(e) (* k_scale for 1-byte caches)
+  float v_scale;                  // 1 for 16/32-bit caches
   // append mode (all non-null) or plain decode (all null): the step's new token
   // rows [S][Hkv][D], written at position context_len - 1 before it is attended
   const void *new_k, *new_v;
@@ -103,6 +103,8 @@ struct FmaMath {
   static constexpr int kPBytes = kDecodeWarps * kBlockSize * G * 4;
   static constexpr int kScratchBytes = kQBytes + kPBytes;
   static constexpr bool kNeedsQInSmem = true;
+  static constexpr int kRowBytes = 256;
+  static constexpr int kStagesPerWarp = pa::kStagesPerWarp;
 
   float m_run[G], l_run[G];
   float2 o[G][EPC / 2];
@@ -208,7 +210,7 @@ struct FmaMath {
   }
 
   // Merge the lane partials and write this warp's (m, l, o) for the G heads.
-  __device__ void write_partials(float *o_s, float *m_s, float *l_s, int warp, int lane) {
+  __device__ void write_partials(float *o_s, float *m_s, float *l_s, int warp, int lane, float) {
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       float l = l_run[hh];   // lanes t and t+16 hold the same p: sum over one half
@@ -309,6 +311,8 @@ struct MmaMath {
   static constexpr int D = 128;
   static constexpr int kScratchBytes = 0;
   static constexpr bool kNeedsQInSmem = false;
+  static constexpr int kRowBytes = 256;
+  static constexpr int kStagesPerWarp = pa::kStagesPerWarp;
 
   // Fragment roles (m16n8k16): gid = lane / 4 is the row group, tig = lane % 4.
   //   S^T / P^T: this lane holds tokens gid and gid+8 for heads 2*tig, 2*tig+1.
@@ -419,7 +423,7 @@ struct MmaMath {
     }
   }
 
-  __device__ void write_partials(float *o_s, float *m_s, float *l_s, int warp, int lane) {
+  __device__ void write_partials(float *o_s, float *m_s, float *l_s, int warp, int lane, float) {
     const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -448,11 +452,183 @@ struct MmaMath {
   }
 };
 
+// ============================================================ tensor-core math, 1-byte E4M3 caches
+// Two E4M3 codes (low byte first) -> f16x2 (low half first); exact: every E4M3
+// value is an f16.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t &lo, uint32_t &hi) {
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n cvt.rn.f16x2.e4m3x2 %1, h;\n}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+__device__ __forceinline__ uint32_t f16x2_from(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Block math for 1-byte E4M3 caches (rows of 128 bytes, head_dim 128), q and
+// out in T (fp16 or bf16).  Same transposed MMA problem as MmaMath, in f16:
+//  * QK: ldmatrix of the code tile gives each lane 4 consecutive codes of one
+//    token; converted they fill the A fragment with head_dim permuted inside
+//    every 16-wide k-step (k-slots 2t,2t+1,2t+8,2t+9 <-> d 4t..4t+3), and the
+//    Q^T fragments use the same permutation.
+//  * PV: ldmatrix.trans of the code tile (16-bit units = code pairs) gives two
+//    tokens x two d; one byte permute makes (token pair at d0 | token pair at
+//    d1), so the V^T A fragment holds rows d = 16c + 2*gid and 16c + 2*gid + 1
+//    (a row permutation of the output tile, undone in write_partials).
+//  * scores carry k_scale (folded into scale_log2), outputs v_scale.
+//  * P is one f16 (relative rounding 2^-12).
+// q is converted to f16 once (exact for |q| in the f16 normal range).
+template <typename T, int G>
+struct Fp8MmaMath {
+  static_assert(G >= 1 && G <= 8, "the N = 8 side holds up to 8 query heads");
+  static constexpr int D = 128;
+  static constexpr int kScratchBytes = 0;
+  static constexpr bool kNeedsQInSmem = false;
+  static constexpr int kRowBytes = 128;
+  static constexpr int kStagesPerWarp = 2 * pa::kStagesPerWarp;   // same bytes in flight as 256-byte rows
+
+  uint32_t qf[8][2];
+  float m_run[2], l_run[2];
+  float o[8][4];
+  int off[4];           // ldmatrix row offsets: chunks 2x, 2x+1 (tokens 0-7, 8-15)
+
+  __device__ static void stage_q(uint8_t *, const T *, float) {}
+
+  __device__ void init(uint8_t *, const T *qg, float, int, int lane) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (gid < G) {
+        const T *q4 = qg + gid * D + 16 * c + 4 * tig;
+        qf[c][0] = f16x2_from(Elem<T>::load(q4), Elem<T>::load(q4 + 1));
+        qf[c][1] = f16x2_from(Elem<T>::load(q4 + 2), Elem<T>::load(q4 + 3));
+      } else {
+        qf[c][0] = qf[c][1] = 0u;
+      }
+    }
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+    const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) off[x] = tile_offset(ri + 8 * (mi & 1), 2 * x + (mi >> 1));
+  }
+
+  __device__ void block(const uint8_t *tk, uint8_t *tv, int nvalid, int lane, float scale_log2) {
+    const int gid = lane >> 2;
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      uint32_t r[4];
+      ldmatrix_x4(r, tk + off[x]);   // r0/r1: chunk 2x tokens 0-7 / 8-15; r2/r3: chunk 2x+1
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        uint32_t a[4];
+        e4m3x4_to_f16x2x2(r[2 * kk], a[0], a[2]);
+        e4m3x4_to_f16x2x2(r[2 * kk + 1], a[1], a[3]);
+        mma_f16(s, a, qf[2 * x + kk][0], qf[2 * x + kk][1]);
+      }
+    }
+    const bool v0 = gid < nvalid, v1 = gid + 8 < nvalid;
+    const float x0 = v0 ? s[0] * scale_log2 : -INFINITY;
+    const float x1 = v0 ? s[1] * scale_log2 : -INFINITY;
+    const float x2 = v1 ? s[2] * scale_log2 : -INFINITY;
+    const float x3 = v1 ? s[3] * scale_log2 : -INFINITY;
+    float mb0 = fmaxf(x0, x2), mb1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int d = 4; d < 32; d <<= 1) {
+      mb0 = fmaxf(mb0, __shfl_xor_sync(kFullMask, mb0, d));
+      mb1 = fmaxf(mb1, __shfl_xor_sync(kFullMask, mb1, d));
+    }
+    const float mn0 = fmaxf(m_run[0], mb0), mn1 = fmaxf(m_run[1], mb1);
+    if (__any_sync(kFullMask, mn0 != m_run[0] || mn1 != m_run[1])) {
+      const float a0 = ex2(m_run[0] - mn0), a1 = ex2(m_run[1] - mn1);
+      l_run[0] *= a0;
+      l_run[1] *= a1;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        o[m][0] *= a0;
+        o[m][1] *= a1;
+        o[m][2] *= a0;
+        o[m][3] *= a1;
+      }
+      m_run[0] = mn0;
+      m_run[1] = mn1;
+    }
+    const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1), p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
+    l_run[0] += p0 + p2;
+    l_run[1] += p1 + p3;
+
+    if (nvalid < kBlockSize) {   // rows past the end: code 0 (+0) so that 0 * V stays 0
+      uint4 *rows = reinterpret_cast<uint4 *>(tv);
+      for (int i = nvalid * 8 + lane; i < kBlockSize * 8; i += 32) rows[i] = make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+    }
+    const uint32_t b0 = movmatrix_trans(f16x2_from(p0, p1));
+    const uint32_t b1 = movmatrix_trans(f16x2_from(p2, p3));
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      uint32_t r[4];
+      ldmatrix_x4_trans(r, tv + off[x]);
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        // (token 2t: d0 d1 | token 2t+1: d0 d1) -> (d0: 2t 2t+1 | d1: 2t 2t+1)
+        const uint32_t lo = __byte_perm(r[2 * kk], 0u, 0x3120);
+        const uint32_t hi = __byte_perm(r[2 * kk + 1], 0u, 0x3120);
+        uint32_t a[4];
+        e4m3x4_to_f16x2x2(lo, a[0], a[1]);
+        e4m3x4_to_f16x2x2(hi, a[2], a[3]);
+        mma_f16(o[2 * x + kk], a, b0, b1);
+      }
+    }
+  }
+
+  __device__ void write_partials(float *o_s, float *m_s, float *l_s, int warp, int lane, float v_scale) {
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float l = l_run[j];
+      l += __shfl_xor_sync(kFullMask, l, 4);
+      l += __shfl_xor_sync(kFullMask, l, 8);
+      l += __shfl_xor_sync(kFullMask, l, 16);
+      l_run[j] = l;
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int hh = 2 * tig + j;
+      if (hh < G) {
+        float *dst = o_s + (warp * G + hh) * D + 2 * gid;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {   // m-tile m rows: d = 16m + 2*gid (c0,c1) and 16m + 2*gid + 1 (c2,c3)
+          dst[16 * m] = o[m][j] * v_scale;
+          dst[16 * m + 1] = o[m][2 + j] * v_scale;
+        }
+        if (gid == 0) {
+          m_s[warp * G + hh] = m_run[j];
+          l_s[warp * G + hh] = l_run[j];
+        }
+      }
+    }
+  }
+};
+
 // ============================================================ shared memory plan
 template <typename T, int G, typename Math>
 struct DecodeSmem {
-  static constexpr int D = kChunksPerRow * Elem<T>::kPerChunk;
-  static constexpr int kTilesBytes = kStages * 2 * kTileBytes;
+  static constexpr int D = Math::D;
+  static constexpr int kTile = kBlockSize * Math::kRowBytes;        // one K or V tile
+  static constexpr int kStages = kDecodeWarps * Math::kStagesPerWarp;
+  static constexpr int kTilesBytes = kStages * 2 * kTile;
   static constexpr int kScratchOff = kTilesBytes;
   static constexpr int kMOff = kScratchOff + Math::kScratchBytes;
   static constexpr int kLOff = kMOff + kDecodeWarps * G * 4;
@@ -470,6 +646,9 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
                                const DecodeParams p) {
   using SM = DecodeSmem<T, G, Math>;
   constexpr int D = SM::D;
+  constexpr int kTile = SM::kTile;
+  constexpr int kStages = SM::kStages;
+  constexpr int kSPW = Math::kStagesPerWarp;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -537,16 +716,17 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
       }
     }
     const int id = __shfl_sync(kFullMask, my_id, j & 31);
-    const int s = warp + (j % kStagesPerWarp) * kDecodeWarps;
+    const int s = warp + (j % kSPW) * kDecodeWarps;
     if (lane == 0) {
       if (id >= 0) {
-        // one box per 128-byte half of the rows: the tile lands as [half][token][128 B]
-        uint8_t *tk = smem + s * 2 * kTileBytes;
-        mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
-        tma_load_5d(tk, &tm_k, 0, 0, g, 0, id, &full[s], policy);
-        tma_load_5d(tk + kTileBytes / 2, &tm_k, 0, 1, g, 0, id, &full[s], policy);
-        tma_load_5d(tk + kTileBytes, &tm_v, 0, 0, g, 0, id, &full[s], policy);
-        tma_load_5d(tk + kTileBytes + kTileBytes / 2, &tm_v, 0, 1, g, 0, id, &full[s], policy);
+        // one box per 128-byte part of the rows: the tile lands as [part][token][128 B]
+        uint8_t *tk = smem + s * 2 * kTile;
+        mbar_arrive_expect_tx(&full[s], 2 * kTile);
+#pragma unroll
+        for (int part = 0; part < Math::kRowBytes / 128; ++part) {
+          tma_load_5d(tk + part * 2048, &tm_k, 0, part, g, 0, id, &full[s], policy);
+          tma_load_5d(tk + kTile + part * 2048, &tm_v, 0, part, g, 0, id, &full[s], policy);
+        }
       } else {
         mbar_arrive(&full[s]);   // bad id: recorded above; complete the phase without data
       }
@@ -556,7 +736,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   if constexpr (Math::kNeedsQInSmem) Math::stage_q(scratch, qg, p.scale_log2);
   __syncthreads();   // barriers initialised (and q staged)
 
-  for (int j = 0; j < min(nw, kStagesPerWarp); ++j) issue(j);
+  for (int j = 0; j < min(nw, kSPW); ++j) issue(j);
 
   Math math;
   math.init(scratch, qg, p.scale_log2, warp, lane);
@@ -564,8 +744,8 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   bool ok = true;
   int j = 0;
   for (; j < nw; ++j) {
-    const int s = warp + (j % kStagesPerWarp) * kDecodeWarps;
-    const bool landed = mbar_wait(&full[s], (j / kStagesPerWarp) & 1);
+    const int s = warp + (j % kSPW) * kDecodeWarps;
+    const bool landed = mbar_wait(&full[s], (j / kSPW) & 1);
     if (!__all_sync(kFullMask, landed)) {
       if (lane == 0) {
         record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, blockIdx.x);
@@ -574,10 +754,10 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
       ok = false;
       break;
     }
-    uint8_t *tk = smem + s * 2 * kTileBytes;
+    uint8_t *tk = smem + s * 2 * kTile;
     const int lb = warp + j * kDecodeWarps;   // local block index
     const int nvalid = min(kBlockSize, tok1 - (tok0 + lb * kBlockSize));
-    if (p.new_k != nullptr && part == nparts - 1 && lb == nblk - 1) {
+    if (Math::kRowBytes == 256 && p.new_k != nullptr && part == nparts - 1 && lb == nblk - 1) {
       // append mode: this block holds position L-1.  Store the new token's K/V
       // rows of head g in the cache and put them into the tile that just landed
       // (its copy of that row may predate the store).  Lanes 0-15 move the 16
@@ -594,26 +774,26 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
                      ((static_cast<size_t>(id) * kBlockSize + t_new) * p.num_kv_heads + g) * kChunksPerRow + c;
         *dst = x;
       }
-      *reinterpret_cast<uint4 *>(tk + (is_v ? kTileBytes : 0) + tile_offset(t_new, c)) = x;
+      *reinterpret_cast<uint4 *>(tk + (is_v ? kTile : 0) + tile_offset(t_new, c)) = x;
       __syncwarp();
     }
-    math.block(tk, tk + kTileBytes, nvalid, lane, p.scale_log2);
+    math.block(tk, tk + kTile, nvalid, lane, p.scale_log2);
     __syncwarp();   // all lanes done with the stage
-    if (j + kStagesPerWarp < nw) {
+    if (j + kSPW < nw) {
       fence_proxy_async_smem();
-      issue(j + kStagesPerWarp);
+      issue(j + kSPW);
     }
   }
   if (!ok) {
     // let this warp's other copies in flight land (bounded) before the CTA can exit
-    for (int jj = j + 1; jj < min(nw, j + kStagesPerWarp); ++jj)
-      mbar_wait(&full[warp + (jj % kStagesPerWarp) * kDecodeWarps], (jj / kStagesPerWarp) & 1);
+    for (int jj = j + 1; jj < min(nw, j + kSPW); ++jj)
+      mbar_wait(&full[warp + (jj % kSPW) * kDecodeWarps], (jj / kSPW) & 1);
   }
 
   // ---- merge the warps through shared memory (the stage tiles are reused)
   __syncthreads();
   float *o_s = reinterpret_cast<float *>(smem);
-  math.write_partials(o_s, m_s, l_s, warp, lane);
+  math.write_partials(o_s, m_s, l_s, warp, lane, p.v_scale);
   __syncthreads();
   if (*abort_s) return;
 

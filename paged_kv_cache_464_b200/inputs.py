@@ -24,6 +24,9 @@ Workloads (sizes, distributions):
                       private suffix U[16,512]; 32/8 heads, D=128; 25% of the
                       sequences copy-on-write the last prefix block.
 * ``long_context``    bf16, 8 seqs, len 32768, 64/8 heads, D=128, partition 512.
+* ``llama3_8b_gqa_fp8``  the GQA workload with an FP8 (E4M3) KV cache: the case
+                      carries bf16 rows; a quantising slot write stores them as
+                      1-byte codes with scale 0.0125 (k and v).
 
 ``context_lens`` are the lengths the decode call attends to.  The step's new
 token sits at position ``context_len - 1``: the pre-step cache holds poison at
@@ -58,6 +61,8 @@ class DecodeConfig:
     block_size: int = 16
     partition_size: int = 0  # 0 = library's automatic choice
     description: str = ""
+    kv_dtype: str = ""       # "" = dtype; "fp8_e4m3": caches hold 1-byte codes written from the dtype rows
+    kv_scale: float = 1.0    # k_scale = v_scale for 1-byte caches
 
     @property
     def seed(self) -> int:
@@ -83,12 +88,15 @@ CONFIGS: Dict[str, DecodeConfig] = {
         DecodeConfig("long_context", 5, 8, 64, 8, 128, "bf16", partition_size=512,
                      description="long-context split-K decode bf16, 8 seqs x 32768, 64/8 heads, "
                                  "D=128, partition 512"),
+        DecodeConfig("llama3_8b_gqa_fp8", 6, 256, 32, 8, 128, "bf16", kv_dtype="fp8_e4m3", kv_scale=0.0125,
+                     description="the Llama-3-8B-shaped GQA workload with an FP8 (E4M3) KV cache: bf16 q/out, "
+                                 "K/V stored as 1-byte codes with scale 0.0125"),
     ]
 }
 
 
-def poison_value(dtype: str) -> float:
-    return float("nan")
+# the workloads whose caches hold the storage dtype itself (the five of the target list)
+BASE_WORKLOADS = [n for n, c in CONFIGS.items() if not c.kv_dtype]
 
 
 def _round(x: np.ndarray, dtype: str) -> torch.Tensor:
@@ -102,7 +110,7 @@ def _draw_lens(cfg: DecodeConfig, rng: np.random.Generator) -> np.ndarray:
         return np.array([17, 33, 50, 100], dtype=np.int64)
     if cfg.name == "llama2_7b":
         return rng.integers(64, 2048, size=S, endpoint=True).astype(np.int64)
-    if cfg.name == "llama3_8b_gqa":
+    if cfg.name in ("llama3_8b_gqa", "llama3_8b_gqa_fp8"):
         x = np.exp(rng.normal(math.log(1024.0), 0.6, size=S))
         return np.clip(np.rint(x), 128, 4096).astype(np.int64)
     if cfg.name == "shared_prefix":
@@ -158,7 +166,8 @@ class DecodeCase:
     def kv_bytes(self) -> int:
         """Algorithmic KV bytes one decode call reads: sum_b L_b * Hkv * 2 * D * es."""
         c = self.cfg
-        return int(self.context_lens.to(torch.int64).sum().item()) * c.num_kv_heads * 2 * c.head_dim * ELEM_BYTES[c.dtype]
+        es = 1 if c.kv_dtype == "fp8_e4m3" else ELEM_BYTES[c.dtype]
+        return int(self.context_lens.to(torch.int64).sum().item()) * c.num_kv_heads * 2 * c.head_dim * es
 
 
 def make_case(name_or_cfg, *, seed: Optional[int] = None, num_seqs: Optional[int] = None,

@@ -80,7 +80,7 @@ def pin_widening(o):
 
 
 def pin_dense_equivalence(o, names=None, tol=1e-12):
-    for name in names or list(inputs.CONFIGS):
+    for name in names or inputs.BASE_WORKLOADS:
         case = small_case(name)
         got = o.decode_case(case)
         ref = sdpa_reference(case)
@@ -214,7 +214,7 @@ def pin_closed_forms(o):
 
 
 def pin_slot_rule(o):
-    for name in inputs.CONFIGS:
+    for name in inputs.BASE_WORKLOADS:
         case = small_case(name)
         L = case.context_lens.numpy()
         for b in range(case.cfg.num_seqs):
@@ -223,7 +223,7 @@ def pin_slot_rule(o):
 
 
 def pin_cache_writes(o):
-    for name in inputs.CONFIGS:
+    for name in inputs.BASE_WORKLOADS:
         case = small_case(name)
         k = case.k_cache.clone()
         v = case.v_cache.clone()

@@ -102,6 +102,7 @@ def test_decode_host_validation(capi):
     assert _decode(capi, maxL=4096, P=512) == PA_ERR_WORKSPACE  # split needs a workspace
     assert _decode(capi, maxL=4096, P=512, ws=256, wsb=10) == PA_ERR_WORKSPACE
     assert _decode(capi, S=0) == 0                              # nothing to do
+    assert _decode(capi, dt=3, D=128) == PA_ERR_DTYPE           # 1-byte caches go through pa_decode_fp8
 
 
 def test_cache_ops_host_validation(capi):
@@ -111,9 +112,27 @@ def test_cache_ops_host_validation(capi):
     assert r.pa_reshape_and_cache(16, 16, 16, 16, 16, -1, 8, 16, 4, 64, 0, None) == 3
     assert r.pa_reshape_and_cache(None, 16, 16, 16, 16, 4, 8, 16, 4, 64, 0, None) == 1
     assert r.pa_reshape_and_cache(16, 16, 24, 16, 16, 4, 8, 16, 4, 64, 0, None) == 6
-    assert r.pa_reshape_and_cache(16, 16, 16, 16, 16, 4, 8, 16, 4, 64, 3, None) == 2
+    assert r.pa_reshape_and_cache(16, 16, 16, 16, 16, 4, 8, 16, 4, 64, 7, None) == 2
+    assert r.pa_reshape_and_cache(16, 16, 16, 16, 16, 4, 8, 16, 4, 64, 3, None) == 3     # 1-byte rows must be 128 B
     # (k_cache, v_cache, mapping, P, NB, bs, Hkv, D, dtype, stream)
     assert r.pa_copy_blocks(16, 16, 16, 0, 8, 16, 4, 64, 0, None) == 0
     assert r.pa_copy_blocks(16, 16, None, 2, 8, 16, 4, 64, 0, None) == 1
     assert r.pa_copy_blocks(16, 16, 16, -2, 8, 16, 4, 64, 0, None) == 3
     assert r.pa_copy_blocks(16, 16, 16, 2, 8, 16, 4, 96, 1, None) == 3
+
+
+def test_fp8_host_validation(capi):
+    r = capi.raw
+    # pa_reshape_and_cache_fp8(key, value, kc, vc, slots, T, NB, bs, Hkv, D, src_dtype, k_scale, v_scale, stream)
+    assert r.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 0, 8, 16, 4, 128, 2, 0.1, 0.1, None) == 0
+    assert r.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 4, 8, 16, 4, 128, 0, 0.1, 0.1, None) == 2   # f32 source
+    assert r.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 4, 8, 16, 4, 64, 2, 0.1, 0.1, None) == 3    # D=64
+    assert r.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 4, 8, 16, 4, 128, 2, 0.0, 0.1, None) == 3   # scale 0
+    assert r.pa_reshape_and_cache_fp8(16, 16, 8, 16, 16, 4, 8, 16, 4, 128, 2, 0.1, 0.1, None) == 6    # alignment
+    # pa_decode_fp8(out, q, kc, vc, ks, vs, bt, mbs, cl, S, Hq, maxL, scale, P, ws, wsb, NB, bs, Hkv, D, q_dtype, s)
+    dec = lambda **k: r.pa_decode_fp8(k.get("out", 16), 16, 16, 16, k.get("ks", 0.1), 0.1, 16, 4, 16, 2, 8, 64,
+                                      0.088, 0, None, 0, 8, 16, 2, k.get("D", 128), k.get("qd", 2), None)
+    assert dec(qd=0) == 2            # q must be fp16 or bf16
+    assert dec(D=64) == 3
+    assert dec(ks=float("inf")) == 3
+    assert dec(out=8) == 6

@@ -89,7 +89,7 @@ SMALL = {
 }
 
 
-@pytest.mark.parametrize("name", list(inputs.CONFIGS))
+@pytest.mark.parametrize("name", inputs.BASE_WORKLOADS)
 def test_step_small(pa, orc, name):
     """copy-on-write copies, new-token write and decode on small cases of every workload."""
     case = inputs.make_case(name, lens=SMALL[name])
@@ -100,7 +100,7 @@ def test_step_small(pa, orc, name):
     assert_decode_close(out, ref, case.cfg.dtype, name)
 
 
-@pytest.mark.parametrize("name", list(inputs.CONFIGS))
+@pytest.mark.parametrize("name", inputs.BASE_WORKLOADS)
 def test_step_full_size(pa, orc, name):
     """Every workload at its full size, all outputs, in the launch configuration the benchmark times."""
     case = inputs.make_case(name, with_post=False)
@@ -262,7 +262,7 @@ def gpu_step_append(pa, case, partition_size=None):
     return out, d
 
 
-@pytest.mark.parametrize("name", list(inputs.CONFIGS))
+@pytest.mark.parametrize("name", inputs.BASE_WORKLOADS)
 def test_append_step_small(pa, orc, name):
     case = inputs.make_case(name, lens=SMALL[name])
     out, d = gpu_step_append(pa, case)
@@ -275,7 +275,7 @@ def test_append_step_small(pa, orc, name):
     assert torch.equal(out.cpu(), out2.cpu())
 
 
-@pytest.mark.parametrize("name", list(inputs.CONFIGS))
+@pytest.mark.parametrize("name", inputs.BASE_WORKLOADS)
 def test_append_step_full_size(pa, orc, name):
     case = inputs.make_case(name, with_post=False)
     out, d = gpu_step_append(pa, case)
