@@ -78,6 +78,8 @@ class Oracle:
                                                      ctypes.c_float]
         lib.oracle_paged_decode_fp8.restype = I
         lib.oracle_paged_decode_fp8.argtypes = [P, P, I, U8, U8, D, D, P, I, P, I, I, I, I, I, I, D]
+        lib.oracle_paged_prefill.restype = I
+        lib.oracle_paged_prefill.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, D, I]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         self.lib = lib
@@ -156,6 +158,25 @@ class Oracle:
         if rc:
             raise OracleError(rc)
         return self.paged_decode(case.q, k, v, case.block_tables, case.context_lens, case.scale)
+
+    # -- prefill -------------------------------------------------------------------------
+    def paged_prefill(self, q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale):
+        """q [T, Hq, D]; chunk of sequence b = rows query_start_loc[b]:query_start_loc[b+1],
+        the last tokens of its context.  Returns out [T, Hq, D] f64."""
+        T, Hq, D = q.shape
+        NB, bs, Hkv, D2 = k_cache.shape
+        assert D2 == D and q.dtype == k_cache.dtype == v_cache.dtype
+        bt = block_tables.to(torch.int32).contiguous()
+        cl = context_lens.to(torch.int32).contiguous()
+        qsl = query_start_loc.to(torch.int32).contiguous()
+        S = cl.numel()
+        out = np.zeros((T, Hq, D), dtype=np.float64)
+        rc = self.lib.oracle_paged_prefill(_ptr(out), _ptr(q.contiguous()), _ptr(k_cache.contiguous()),
+                                           _ptr(v_cache.contiguous()), _ptr(bt), bt.shape[1], _ptr(cl), _ptr(qsl), S,
+                                           Hq, Hkv, D, bs, NB, float(np.float32(scale)), DTYPE_CODE[q.dtype])
+        if rc:
+            raise OracleError(rc)
+        return out
 
     # -- FP8 (E4M3) caches ------------------------------------------------------------
     def e4m3_decode(self, codes: torch.Tensor) -> np.ndarray:

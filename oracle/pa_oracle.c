@@ -56,6 +56,8 @@
  *                            inside the finite range; saturation outside it.
  *   oracle_reshape_and_cache_fp8  the slot layout of oracle_reshape_and_cache.
  *   oracle_paged_decode_fp8  torch SDPA (fp64) on the dequantised logical K/V.
+ *   oracle_paged_prefill     torch SDPA (fp64) with the causal mask at the
+ *                            chunk's offset; later tokens do not matter.
  */
 #include <math.h>
 #include <stdint.h>
@@ -458,6 +460,88 @@ int oracle_paged_decode_fp8(double *out, const void *q, int q_dtype, const uint8
       int32_t physical_block = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
       int64_t row = (((int64_t)physical_block * block_size + t % block_size) * num_kv_heads + g) * D;
       for (int64_t d = 0; d < D; ++d) o[d] += s[t] * (e4m3_value(v_cache[row + d]) * v_scale);
+    }
+    free(s);
+    free(qv);
+  }
+  return status;
+}
+
+/*
+ * Paged prefill (a chunk of new tokens per sequence attending, causally, to the
+ * sequence's cached tokens through its block table).  The pages' engine runs
+ * prompts in chunks ("vLLM推理引擎深度实战：…" §五 / tuning: enable_chunked_prefill);
+ * the attention of each new token is [A] §五's formula with the context cut at
+ * that token.  Reading: sequence b's chunk holds n_b = query_start_loc[b+1] -
+ * query_start_loc[b] queries, which are the last n_b of its context_lens[b]
+ * tokens (their K/V are already in the cache); query i sits at position
+ * p = L_b - n_b + i and attends to tokens 0..p.
+ *
+ * q, out: [T][Hq][D] with T = query_start_loc[num_seqs]; out double.
+ */
+int oracle_paged_prefill(double *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                         const int32_t *query_start_loc, int num_seqs, int num_heads, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, double scale, int dtype) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_heads % num_kv_heads != 0)
+    return ORACLE_BAD_ARGS;
+  const int group = num_heads / num_kv_heads;
+  const int64_t D = head_dim;
+  for (int b = 0; b < num_seqs; ++b) {
+    int L = context_lens[b];
+    int n = query_start_loc[b + 1] - query_start_loc[b];
+    if (n < 0 || L < n || (int64_t)L > (int64_t)max_blocks_per_seq * block_size) return ORACLE_BAD_CONTEXT_LEN;
+    for (int j = 0; j < (L + block_size - 1) / block_size; ++j) {
+      int32_t id = block_tables[(int64_t)b * max_blocks_per_seq + j];
+      if (id < 0 || id >= num_blocks) return ORACLE_BAD_BLOCK_ID;
+    }
+  }
+  const int64_t T = query_start_loc[num_seqs];
+  int status = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < T * num_heads; ++r) {
+    const int64_t tok = r / num_heads;
+    const int h = (int)(r % num_heads);
+    int b = 0;
+    while (query_start_loc[b + 1] <= tok) ++b;
+    const int L = context_lens[b];
+    const int n = query_start_loc[b + 1] - query_start_loc[b];
+    const int pos = L - n + (int)(tok - query_start_loc[b]);   /* this query's position */
+    const int g = h / group;
+    const int len = pos + 1;                                    /* tokens 0..pos */
+    double *o = out + r * D;
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    double *s = (double *)malloc(sizeof(double) * (size_t)len);
+    double *qv = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!s || !qv) {
+      free(s);
+      free(qv);
+#pragma omp atomic write
+      status = ORACLE_NO_MEMORY;
+      continue;
+    }
+    for (int64_t d = 0; d < D; ++d) qv[d] = widen_one(q, r * D + d, dtype);
+    for (int t = 0; t < len; ++t) {
+      int32_t physical_block = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
+      int64_t row = (((int64_t)physical_block * block_size + t % block_size) * num_kv_heads + g) * D;
+      double dot = 0.0;
+      for (int64_t d = 0; d < D; ++d) dot += qv[d] * widen_one(k_cache, row + d, dtype);
+      s[t] = scale * dot;
+    }
+    double m = s[0];
+    for (int t = 1; t < len; ++t)
+      if (s[t] > m) m = s[t];
+    double z = 0.0;
+    for (int t = 0; t < len; ++t) {
+      s[t] = exp(s[t] - m);
+      z += s[t];
+    }
+    for (int t = 0; t < len; ++t) s[t] = s[t] / z;
+    for (int t = 0; t < len; ++t) {
+      int32_t physical_block = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
+      int64_t row = (((int64_t)physical_block * block_size + t % block_size) * num_kv_heads + g) * D;
+      for (int64_t d = 0; d < D; ++d) o[d] += s[t] * widen_one(v_cache, row + d, dtype);
     }
     free(s);
     free(qv);

@@ -344,3 +344,74 @@ def permute_blocks(case: DecodeCase, seed: int) -> DecodeCase:
         k_cache_post=move(case.k_cache_post), v_cache_post=move(case.v_cache_post),
         block_tables=retab(case.block_tables), shared_block_tables=retab(case.shared_block_tables),
         slot_mapping=new_sm, block_mapping=new_bm)
+
+
+# ---------------------------------------------------------------------------- prefill
+@dataclasses.dataclass
+class PrefillCase:
+    """A chunk of new tokens per sequence over a paged cache (all tokens already cached).
+
+    q                [T, Hq, D]   the chunk tokens' queries, sequence after sequence
+    query_start_loc  [S + 1] int32   sequence b's queries are rows qsl[b]:qsl[b+1];
+                                     they are the last n_b tokens of its context
+    k_cache, v_cache [NB, bs, Hkv, D]  every context token present
+    """
+    cfg: DecodeConfig
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_tables: torch.Tensor
+    context_lens: torch.Tensor
+    query_start_loc: torch.Tensor
+    scale: float
+    k_logical: Optional[List[np.ndarray]] = None
+    v_logical: Optional[List[np.ndarray]] = None
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start_loc[-1])
+
+    @property
+    def max_query_len(self) -> int:
+        q = self.query_start_loc
+        return int((q[1:] - q[:-1]).max()) if len(q) > 1 else 0
+
+    def flops(self) -> int:
+        """Multiply-add flops of S = QK^T and O = PV over the causally visible keys."""
+        c = self.cfg
+        L = self.context_lens.to(torch.int64)
+        n = (self.query_start_loc[1:] - self.query_start_loc[:-1]).to(torch.int64)
+        visible = (n * (L - n) + n * (n + 1) // 2).sum().item()   # sum over queries of (position + 1)
+        return int(4 * visible * c.num_heads * c.head_dim)
+
+
+PREFILL_CONFIGS: Dict[str, DecodeConfig] = {
+    c.name: c for c in [
+        DecodeConfig("llama3_8b_prefill", 7, 16, 32, 8, 128, "bf16",
+                     description="Llama-3-8B-shaped chunked prefill bf16: 16 sequences, 512-token chunks "
+                                 "after a cached prefix U[0,1536], 32/8 heads, D=128"),
+    ]
+}
+
+
+def make_prefill_case(name_or_cfg, *, chunk_lens=None, prefix_lens=None, seed=None,
+                      keep_logical: bool = False) -> PrefillCase:
+    """Context = prefix + chunk per sequence; every context token is drawn and
+    placed in the cache (through make_case); q is drawn for the chunk tokens."""
+    cfg = PREFILL_CONFIGS[name_or_cfg] if isinstance(name_or_cfg, str) else name_or_cfg
+    rng = np.random.Generator(np.random.PCG64(cfg.seed if seed is None else seed))
+    S = cfg.num_seqs if chunk_lens is None else len(chunk_lens)
+    if chunk_lens is None:
+        chunk_lens = [512] * S
+    if prefix_lens is None:
+        prefix_lens = rng.integers(0, 1536, size=S, endpoint=True).tolist()
+    L = [int(a) + int(b) for a, b in zip(prefix_lens, chunk_lens)]
+    base = make_case(dataclasses.replace(cfg, num_seqs=S), lens=L, seed=int(rng.integers(1 << 31)),
+                     keep_logical=keep_logical)
+    T = int(sum(chunk_lens))
+    q = _round(rng.standard_normal((T, cfg.num_heads, cfg.head_dim), dtype=np.float32), cfg.dtype)
+    qsl = torch.zeros(S + 1, dtype=torch.int32)
+    qsl[1:] = torch.cumsum(torch.tensor(chunk_lens, dtype=torch.int32), 0)
+    return PrefillCase(cfg=dataclasses.replace(cfg, num_seqs=S), q=q, k_cache=base.k_cache_post,
+                       v_cache=base.v_cache_post, block_tables=base.block_tables, context_lens=base.context_lens,
+                       query_start_loc=qsl, scale=base.scale, k_logical=base.k_logical, v_logical=base.v_logical)

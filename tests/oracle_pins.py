@@ -382,7 +382,61 @@ def pin_fp8_decode_vs_sdpa(o):
         assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max()), f"{name}: fp8 decode vs SDPA"
 
 
+# ---------------------------------------------------------------------------- prefill
+def _prefill_sdpa(case):
+    c = case.cfg
+    out = np.zeros((case.num_tokens, c.num_heads, c.head_dim))
+    for b in range(c.num_seqs):
+        q0, q1 = int(case.query_start_loc[b]), int(case.query_start_loc[b + 1])
+        n, L = q1 - q0, int(case.context_lens[b])
+        if n == 0:
+            continue
+        K = torch.from_numpy(case.k_logical[b]).permute(1, 0, 2)[None]
+        V = torch.from_numpy(case.v_logical[b]).permute(1, 0, 2)[None]
+        qb = case.q[q0:q1].to(torch.float64).permute(1, 0, 2)[None]         # [1, Hq, n, D]
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]  # query i sees tokens <= L-n+i
+        o = F.scaled_dot_product_attention(qb, K, V, attn_mask=mask, scale=float(np.float32(case.scale)),
+                                           enable_gqa=True)
+        out[q0:q1] = o[0].permute(1, 0, 2).numpy()
+    return out
+
+
+def pin_prefill_vs_sdpa(o):
+    cfg = inputs.PREFILL_CONFIGS["llama3_8b_prefill"]
+    for chunks, prefixes in (([5, 16, 17, 1, 40], [0, 3, 31, 100, 0]), ([64, 33], [200, 1])):
+        case = inputs.make_prefill_case(cfg, chunk_lens=chunks, prefix_lens=prefixes, keep_logical=True)
+        got = o.paged_prefill(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.query_start_loc, case.scale)
+        ref = _prefill_sdpa(case)
+        assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max()), "prefill vs SDPA with causal mask"
+
+
+def pin_prefill_causality(o):
+    cfg = inputs.PREFILL_CONFIGS["llama3_8b_prefill"]
+    case = inputs.make_prefill_case(cfg, chunk_lens=[20], prefix_lens=[30])
+    a = o.paged_prefill(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                        case.query_start_loc, case.scale)
+    k, v = case.k_cache.clone(), case.v_cache.clone()
+    last = int(case.context_lens[0]) - 1
+    blk, off = int(case.block_tables[0, last // 16]), last % 16
+    k[blk, off] = -k[blk, off]
+    v[blk, off] = v[blk, off] + 1
+    b = o.paged_prefill(case.q, k, v, case.block_tables, case.context_lens, case.query_start_loc, case.scale)
+    assert np.array_equal(a[:-1], b[:-1]), "earlier queries must not see a later token"
+    assert not np.array_equal(a[-1], b[-1]), "the last query sees the last token"
+
+
+def pin_prefill_one_query_is_decode(o):
+    cfg = inputs.PREFILL_CONFIGS["llama3_8b_prefill"]
+    case = inputs.make_prefill_case(cfg, chunk_lens=[1, 1, 1], prefix_lens=[0, 16, 700])
+    a = o.paged_prefill(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                        case.query_start_loc, case.scale)
+    b = o.paged_decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale)
+    assert np.array_equal(a, b)
+
+
 ALL_PINS = [pin_widening, pin_dense_equivalence, pin_gqa_mapping, pin_block_permutation,
             pin_length_one, pin_weights, pin_closed_forms, pin_slot_rule, pin_cache_writes,
             pin_copy_blocks, pin_copy_on_write_invariant, pin_errors, pin_e4m3_decode, pin_e4m3_quantize,
-            pin_fp8_cache_layout, pin_fp8_decode_vs_sdpa]
+            pin_fp8_cache_layout, pin_fp8_decode_vs_sdpa, pin_prefill_vs_sdpa, pin_prefill_causality,
+            pin_prefill_one_query_is_decode]

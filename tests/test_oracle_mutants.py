@@ -21,8 +21,8 @@ MUTANTS = [
     ("min_for_max", "if (s[t] > m) m = s[t];\n    double z = 0.0;\n    for (int t = 0; t < L; ++t) {\n      s[t] = exp(s[t] - m);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)",
      "if (s[t] < m) m = s[t];\n    double z = 0.0;\n    for (int t = 0; t < L; ++t) {\n      s[t] = exp(s[t] - m);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)"),
     ("no_normalisation", "for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)", "for (int t = 0; t < L; ++t) s[t] = s[t];\n    if (weights)"),
-    ("value_from_key_cache", "o[d] += s[t] * widen_one(v_cache, row + d, dtype);",
-     "o[d] += s[t] * widen_one(k_cache, row + d, dtype);"),
+    ("value_from_key_cache", '/* out = sum_t w_t * V_t, V_t gathered through the block table */\n    for (int t = 0; t < L; ++t) {\n      int32_t physical_block = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];\n      int offset = t % block_size;\n      int64_t row = (((int64_t)physical_block * block_size + offset) * num_kv_heads + g) * D;\n      for (int64_t d = 0; d < D; ++d) o[d] += s[t] * widen_one(v_cache, row + d, dtype);',
+     '/* out = sum_t w_t * V_t, V_t gathered through the block table */\n    for (int t = 0; t < L; ++t) {\n      int32_t physical_block = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];\n      int offset = t % block_size;\n      int64_t row = (((int64_t)physical_block * block_size + offset) * num_kv_heads + g) * D;\n      for (int64_t d = 0; d < D; ++d) o[d] += s[t] * widen_one(k_cache, row + d, dtype);'),
     ("kv_head_zero", "int64_t row = (((int64_t)physical_block * block_size + offset) * num_kv_heads + g) * D;\n      double dot",
      "int64_t row = (((int64_t)physical_block * block_size + offset) * num_kv_heads + 0) * D;\n      double dot"),
     ("offset_off_by_one", "int offset = t % block_size;\n      int64_t row = (((int64_t)physical_block * block_size + offset) * num_kv_heads + g) * D;\n      double dot",
@@ -43,6 +43,9 @@ MUTANTS = [
      "if (slot < 0) slot = 0;\n    if (slot >= (int64_t)num_blocks * block_size) {\n      if (status == ORACLE_OK) status = ORACLE_BAD_SLOT;\n      continue;\n    }\n    int64_t block = slot / block_size;\n    int64_t offset = slot % block_size;\n    for (int h = 0; h < num_kv_heads; ++h) {\n      int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * row_bytes;"),
     ("weights_without_max_shift", "s[t] = exp(s[t] - m);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)",
      "s[t] = exp(s[t]);\n      z += s[t];\n    }\n    for (int t = 0; t < L; ++t) s[t] = s[t] / z;\n    if (weights)"),
+    ("prefill_causal_off_by_one", "const int len = pos + 1;", "const int len = pos;"),
+    ("prefill_no_offset", "const int pos = L - n + (int)(tok - query_start_loc[b]);",
+     "const int pos = (int)(tok - query_start_loc[b]);"),
     ("e4m3_bias", "v = ldexp(8.0 + m, e - 10);", "v = ldexp(8.0 + m, e - 9);"),
     ("e4m3_ties_to_odd", "(d == best_d && (c & 1) == 0)", "(d == best_d && (c & 1) == 1)"),
     ("e4m3_no_saturation", "if (a >= 448.0) return (uint8_t)(sign ? 0xFE : 0x7E);", "if (a >= 1e30) return 0;"),
