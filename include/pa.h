@@ -1,6 +1,6 @@
 /*
- * pa.h -- C ABI of libpa_b200.so: paged-KV decode attention on NVIDIA B200
- * (sm_100a).
+ * pa.h -- C ABI of libpa_b200.so: paged-KV decode (and chunked-prefill)
+ * attention on NVIDIA B200 (sm_100a).
  *
  * The library implements the decode-time hot path of a paged KV cache as
  * described by these web pages (cited by title and section):
@@ -14,7 +14,8 @@
  *       block map); Block 管理器 (block table per request, block size 16 by
  *       default, copy-on-write of a shared block).
  *   [C] "vLLM推理引擎深度实战：…" §1.2 PagedAttention原理 (block table, allocation
- *       failure reported as an error).
+ *       failure reported as an error); §5.3 推理优化配置 and §7.1 性能调优指南
+ *       (chunked prefill).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -208,6 +209,40 @@ pa_status_t pa_decode_append(void *out, const void *q, const void *key, const vo
                              float scale, int partition_size, void *workspace, size_t workspace_bytes,
                              int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
                              pa_dtype_t dtype, void *stream);
+
+/*
+ * pa_prefill -- paged chunked-prefill attention ([C] §5.3 推理优化配置 and
+ * §7.1 性能调优指南: the engine runs prompts in chunks, enable_chunked_prefill;
+ * each token's attention is [A] §五's formula with the context cut at that
+ * token).
+ *
+ * Sequence b's chunk is the query rows query_start_loc[b] ..
+ * query_start_loc[b+1] - 1 of q; they are the LAST n_b = query_start_loc[b+1] -
+ * query_start_loc[b] tokens of its L_b = context_lens[b] tokens, all of which
+ * (chunk included) are already in the caches (pa_reshape_and_cache).  Query i
+ * of the chunk is position pos = L_b - n_b + i; for each query head h
+ *   out[row, h] = sum_{t <= pos} softmax_t(scale * q[row, h] . K_t[h / G]) V_t[h / G]
+ * with K_t / V_t found through block_tables[b] as in pa_decode, G = num_heads /
+ * num_kv_heads.
+ *
+ * q, out            [T][num_heads][head_dim], T = query_start_loc[num_seqs],
+ *                   dtype PA_F16 or PA_BF16 (= the cache dtype), 16-byte aligned.
+ * query_start_loc   [num_seqs + 1] int32, non-decreasing from 0.
+ * max_query_len     an upper bound of every n_b (sizes the grid).
+ * Other arguments as pa_decode.  head_dim must be 128 and G one of 1, 2, 4, 8.
+ * Computed on the tensor cores (tcgen05) with fp32 accumulation; the softmax
+ * weights enter P V as two 16-bit parts (hi + lo), so accuracy is that of
+ * pa_decode.  Device-side errors: PA_DEV_BAD_CONTEXT_LEN (n_b < 0, n_b >
+ * max_query_len, L_b < n_b or L_b > max_blocks_per_seq * 16: sequence skipped),
+ * PA_DEV_BAD_BLOCK_ID (the block reads as zeros), PA_DEV_WAIT_TIMEOUT.
+ * Errors: PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_CUDA.
+ * num_seqs == 0 or max_query_len == 0 is a no-op.
+ */
+pa_status_t pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                       const int32_t *query_start_loc, int num_seqs, int num_heads, int max_query_len,
+                       float scale, int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                       pa_dtype_t dtype, void *stream);
 
 /*
  * pa_copy_blocks -- copy-on-write block copies ([B] Block 管理器, item 3:

@@ -39,6 +39,8 @@ _lib.pa_reshape_and_cache_fp8.argtypes = [_P, _P, _P, _P, _P, _I, _I64, _I, _I, 
 _lib.pa_decode_fp8.restype = _I
 _lib.pa_decode_fp8.argtypes = [_P, _P, _P, _P, _F, _F, _P, _I, _P, _I, _I, _I, _F, _I, _P, _SZ, _I64, _I, _I, _I, _I,
                                _P]
+_lib.pa_prefill.restype = _I
+_lib.pa_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _I64, _I, _I, _I, _I, _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I64, _I, _I, _I, _I, _P]
 _lib.pa_get_device_error.restype = _I
@@ -47,7 +49,8 @@ _lib.pa_status_string.restype = ctypes.c_char_p
 _lib.pa_status_string.argtypes = [_I]
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_append", "pa_decode_static_workspace", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
+            "pa_decode_append", "pa_decode_static_workspace", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_prefill",
+            "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
 STATIC_WORKSPACE_BYTES = 64 << 20   # PA_STATIC_WORKSPACE_BYTES in include/pa.h
 
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
@@ -273,6 +276,37 @@ def decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_
                               block_tables.shape[1], _dev(context_lens, "context_lens"), S, hq, max_context_len,
                               float(scale), partition_size, ws_ptr, ws_bytes, nb, bs, hkv, d, DTYPE_CODE[q.dtype],
                               _stream(stream)), "pa_decode_fp8")
+    return out
+
+
+def prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+            context_lens: torch.Tensor, query_start_loc: torch.Tensor, scale: float,
+            out: Optional[torch.Tensor] = None, *, max_query_len: Optional[int] = None,
+            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Paged chunked-prefill attention.  q [T, Hq, 128]; sequence b's chunk is rows
+    query_start_loc[b]:query_start_loc[b+1] (int32 [S+1]), the last tokens of its
+    context_lens[b] cached tokens.  ``max_query_len`` (the longest chunk) should be
+    passed by callers that know it; reading it here costs a device-to-host sync."""
+    nb, bs, hkv, d, dt = _cache_args(k_cache, v_cache)
+    T, hq, dq = q.shape
+    if dq != d or q.dtype != k_cache.dtype:
+        raise ValueError("q must be [T, num_heads, head_dim] with the cache dtype")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or query_start_loc.dtype != torch.int32:
+        raise ValueError("block_tables, context_lens and query_start_loc must be int32")
+    S = context_lens.numel()
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or query_start_loc.numel() != S + 1:
+        raise ValueError("block_tables must be [S, MBS] and query_start_loc [S + 1]")
+    if max_query_len is None:
+        qsl = query_start_loc.cpu()
+        max_query_len = int((qsl[1:] - qsl[:-1]).max()) if S else 0
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    _check(_lib.pa_prefill(_dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                           _dev(block_tables, "block_tables"), block_tables.shape[1],
+                           _dev(context_lens, "context_lens"), _dev(query_start_loc, "query_start_loc"), S, hq,
+                           int(max_query_len), float(scale), nb, bs, hkv, d, dt, _stream(stream)), "pa_prefill")
     return out
 
 

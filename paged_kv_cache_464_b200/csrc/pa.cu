@@ -1,6 +1,6 @@
 // pa.cu -- the C ABI of libpa_b200.so (declared in include/pa.h): host-side
 // argument checks, TMA descriptor encoding and kernel launches.  The kernels
-// themselves live in pa_cache_ops.cuh and pa_decode.cuh, compiled here as one
+// themselves live in pa_cache_ops.cuh, pa_decode.cuh and pa_prefill.cuh, compiled here as one
 // translation unit so that the per-device error word needs no separate
 // device linking.
 #include <cudaTypedefs.h>
@@ -15,6 +15,7 @@
 #include "pa.h"
 #include "pa_cache_ops.cuh"
 #include "pa_decode.cuh"
+#include "pa_prefill.cuh"
 
 #ifndef PA_PROGRAMMATIC_LAUNCH
 #define PA_PROGRAMMATIC_LAUNCH 1
@@ -382,6 +383,69 @@ pa_status_t pa_decode_append(void *out, const void *q, const void *key, const vo
   return decode_impl(out, q, key, value, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                      num_seqs, num_heads, max_context_len, scale, partition_size, workspace, workspace_bytes,
                      num_blocks, block_size, num_kv_heads, head_dim, dtype, stream, dtype, 1.f, 1.f);
+}
+
+pa_status_t pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                       const int32_t *query_start_loc, int num_seqs, int num_heads, int max_query_len,
+                       float scale, int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                       pa_dtype_t dtype, void *stream) {
+  pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
+  if (st != PA_OK) return st;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (head_dim != 128 || num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_kv_heads > 65535 ||
+      num_heads % num_kv_heads != 0 || max_query_len < 0 || max_blocks_per_seq < 0 || !std::isfinite(scale))
+    return PA_ERR_SHAPE;
+  const int group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_SHAPE;
+  if ((long long)max_blocks_per_seq * kBlockSize > INT32_MAX) return PA_ERR_SHAPE;
+  if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !context_lens || !query_start_loc || (max_blocks_per_seq > 0 && !block_tables))
+    return PA_ERR_NULL;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
+    return PA_ERR_ALIGN;
+  CUtensorMap mk, mv;
+  if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, kRowBytes) ||
+      !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, kRowBytes))
+    return PA_ERR_CUDA;
+  pa::PrefillParams p{};
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.query_start_loc = query_start_loc;
+  p.num_blocks = num_blocks;
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_query_len = max_query_len;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  const int qt = pa::kPrefillRows / group;   // queries per CTA
+  const dim3 grid((unsigned)((max_query_len + qt - 1) / qt), (unsigned)num_kv_heads, (unsigned)num_seqs);
+  auto go = [&](auto kernel) -> pa_status_t {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pa::PrefillSmem::kAlloc) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    return launch(kernel, grid, dim3(pa::kPrefillThreads), pa::PrefillSmem::kAlloc, (cudaStream_t)stream, mk, mv, p);
+  };
+  if (dtype == PA_BF16) {
+    switch (group) {
+      case 1: return go(pa::pa_prefill_kernel<__nv_bfloat16, 1>);
+      case 2: return go(pa::pa_prefill_kernel<__nv_bfloat16, 2>);
+      case 4: return go(pa::pa_prefill_kernel<__nv_bfloat16, 4>);
+      case 8: return go(pa::pa_prefill_kernel<__nv_bfloat16, 8>);
+    }
+  } else {
+    switch (group) {
+      case 1: return go(pa::pa_prefill_kernel<__half, 1>);
+      case 2: return go(pa::pa_prefill_kernel<__half, 2>);
+      case 4: return go(pa::pa_prefill_kernel<__half, 4>);
+      case 8: return go(pa::pa_prefill_kernel<__half, 8>);
+    }
+  }
+  return PA_ERR_SHAPE;
 }
 
 pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,

@@ -95,6 +95,16 @@ __device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
+// Same, with the default L2 policy (data that other CTAs read again).
+__device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                            int c4, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // L2 policy for data read exactly once (the KV stream).
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

@@ -415,3 +415,17 @@ def make_prefill_case(name_or_cfg, *, chunk_lens=None, prefix_lens=None, seed=No
     return PrefillCase(cfg=dataclasses.replace(cfg, num_seqs=S), q=q, k_cache=base.k_cache_post,
                        v_cache=base.v_cache_post, block_tables=base.block_tables, context_lens=base.context_lens,
                        query_start_loc=qsl, scale=base.scale, k_logical=base.k_logical, v_logical=base.v_logical)
+
+
+def prefill_subcase(case: PrefillCase, seqs: List[int]) -> PrefillCase:
+    """The sequences `seqs` of a prefill case over the same caches (for sampled checks)."""
+    qsl = case.query_start_loc
+    rows = [torch.arange(int(qsl[b]), int(qsl[b + 1])) for b in seqs]
+    lens = torch.tensor([int(qsl[b + 1] - qsl[b]) for b in seqs], dtype=torch.int32)
+    new_qsl = torch.zeros(len(seqs) + 1, dtype=torch.int32)
+    new_qsl[1:] = torch.cumsum(lens, 0)
+    idx = torch.tensor(seqs, dtype=torch.long)
+    return dataclasses.replace(
+        case, cfg=dataclasses.replace(case.cfg, num_seqs=len(seqs)), q=case.q[torch.cat(rows)].contiguous(),
+        block_tables=case.block_tables[idx].contiguous(), context_lens=case.context_lens[idx].contiguous(),
+        query_start_loc=new_qsl, k_logical=None, v_logical=None)

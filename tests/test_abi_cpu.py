@@ -136,3 +136,24 @@ def test_fp8_host_validation(capi):
     assert dec(D=64) == 3
     assert dec(ks=float("inf")) == 3
     assert dec(out=8) == 6
+
+
+def test_prefill_host_validation(capi):
+    r = capi.raw
+    # pa_prefill(out, q, kc, vc, bt, mbs, cl, qsl, S, Hq, max_query_len, scale, NB, bs, Hkv, D, dtype, stream)
+    def pf(**k):
+        a = dict(out=16, q=16, bt=16, mbs=8, cl=16, qsl=16, S=2, Hq=32, mq=64, scale=0.088, bs=16, Hkv=8, D=128,
+                 dt=2)
+        a.update(k)
+        return r.pa_prefill(a["out"], a["q"], 16, 16, a["bt"], a["mbs"], a["cl"], a["qsl"], a["S"], a["Hq"],
+                            a["mq"], a["scale"], 64, a["bs"], a["Hkv"], a["D"], a["dt"], None)
+    assert pf(S=0) == 0 and pf(mq=0) == 0          # nothing to do
+    assert pf(dt=0, D=64) == 2                     # fp32 caches: decode only
+    assert pf(dt=7) == 2
+    assert pf(D=64) == 3                           # head_dim 128 only
+    assert pf(Hq=48) == 3                          # group 6
+    assert pf(Hq=30) == 3                          # Hq % Hkv
+    assert pf(mq=-1) == 3 and pf(S=-1) == 3 and pf(S=70000) == 3
+    assert pf(scale=float("nan")) == 3
+    assert pf(qsl=None) == 1 and pf(q=None) == 1
+    assert pf(out=8) == 6 and pf(qsl=2) == 6
