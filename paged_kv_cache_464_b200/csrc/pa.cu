@@ -394,7 +394,8 @@ pa_status_t pa_prefill(void *out, const void *q, const void *k_cache, const void
   if (st != PA_OK) return st;
   if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
   if (head_dim != 128 || num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_kv_heads > 65535 ||
-      num_heads % num_kv_heads != 0 || max_query_len < 0 || max_blocks_per_seq < 0 || !std::isfinite(scale))
+      num_heads % num_kv_heads != 0 || max_query_len < 0 || max_blocks_per_seq < 0 || !std::isfinite(scale) ||
+      !(scale > 0.f))
     return PA_ERR_SHAPE;
   const int group = num_heads / num_kv_heads;
   if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_SHAPE;
@@ -422,7 +423,7 @@ pa_status_t pa_prefill(void *out, const void *q, const void *k_cache, const void
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.max_query_len = max_query_len;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  const int qt = pa::kPrefillRows / group;   // queries per CTA
+  const int qt = pa::kPrefillTiles * pa::kPrefillRows / group;   // chunk queries per CTA
   const dim3 grid((unsigned)((max_query_len + qt - 1) / qt), (unsigned)num_kv_heads, (unsigned)num_seqs);
   auto go = [&](auto kernel) -> pa_status_t {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pa::PrefillSmem::kAlloc) !=
