@@ -18,6 +18,12 @@ workload) and prints the same kind of line.
 Multi-GPU (torchrun): every rank decodes its own batch of the same shape
 (seed offset by rank); there is no exchange on the data path; the step time is
 the maximum over ranks.
+
+``--workload llama3_8b_prefill`` measures paged chunked prefill instead: a step
+writes the chunk tokens' K/V into their slots (pa_reshape_and_cache) and runs
+pa_prefill (16 sequences, 512-token chunks after cached prefixes of 0..1536
+tokens, 32 query / 8 KV heads, head dim 128, bf16); the metric is attention
+TFLOP/s over the causally visible (query, key) pairs.
 """
 from __future__ import annotations
 
@@ -39,6 +45,8 @@ import torch  # noqa: E402
 from paged_kv_cache_464_b200 import inputs  # noqa: E402
 
 METRIC = "paged decode attention: KV-read GB/s (% of B200 HBM peak), seqs/s"
+PREFILL_METRIC = "paged chunked-prefill attention: TFLOP/s (% of B200 bf16 tensor peak)"
+FALLBACK_BF16_TFLOPS = 1590.0
 DEFAULT_WORKLOAD = "llama3_8b_gqa"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
@@ -59,11 +67,21 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes (read + write) per decode call from the committed ncu summary,
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (a prefill step is well under a second)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def profiled_traffic(workload: str, kernel: str = "pa_decode"):
+    """DRAM bytes (read + write) per call of `kernel` from the committed ncu summary,
     or None when there is none or the kernel sources changed since it was taken."""
     from paged_kv_cache_464_b200 import build
-    path = os.path.join(ROOT, "profiles", f"pa_decode_{workload}.json")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
     try:
         with open(path) as f:
             d = json.load(f)
@@ -392,6 +410,251 @@ def run_ours(args, world, rank, local):
     return line
 
 
+# ------------------------------------------------------------------ chunked prefill
+class PrefillStep:
+    """Device buffers of a chunked-prefill batch; a step writes the chunk tokens'
+    K/V rows into their slots and runs paged prefill attention."""
+
+    def __init__(self, case: inputs.PrefillCase, device):
+        from paged_kv_cache_464_b200 import capi
+        self.pa = capi
+        self.case = case
+        NB, bs, Hkv, D = case.k_cache.shape
+        self.slots_host = chunk_slots(case)
+        self.key_host = case.k_cache.view(NB * bs, Hkv, D)[self.slots_host].contiguous()
+        self.value_host = case.v_cache.view(NB * bs, Hkv, D)[self.slots_host].contiguous()
+        self.q = case.q.to(device)
+        self.kc, self.vc = case.k_cache.to(device), case.v_cache.to(device)
+        self.bt, self.cl = case.block_tables.to(device), case.context_lens.to(device)
+        self.qsl = case.query_start_loc.to(device)
+        self.key, self.value = self.key_host.to(device), self.value_host.to(device)
+        self.slots = self.slots_host.to(device)
+        self.out = torch.empty_like(self.q)
+        self.max_query_len = case.max_query_len
+
+    def write(self):
+        self.pa.reshape_and_cache(self.key, self.value, self.kc, self.vc, self.slots)
+
+    def attend(self):
+        self.pa.prefill(self.q, self.kc, self.vc, self.bt, self.cl, self.qsl, self.case.scale, self.out,
+                        max_query_len=self.max_query_len)
+
+    def __call__(self):
+        self.write()
+        self.attend()
+
+
+def chunk_slots(case: inputs.PrefillCase) -> torch.Tensor:
+    """Slots of every chunk token (positions L - n .. L - 1 of each sequence), in query order."""
+    bs = case.k_cache.shape[1]
+    out = []
+    for b in range(case.cfg.num_seqs):
+        L = int(case.context_lens[b])
+        n = int(case.query_start_loc[b + 1] - case.query_start_loc[b])
+        pos = torch.arange(L - n, L)
+        out.append(case.block_tables[b, pos // bs].to(torch.int64) * bs + pos % bs)
+    return torch.cat(out) if out else torch.zeros(0, dtype=torch.int64)
+
+
+def run_prefill(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    sampler = ClockSampler(local).start()
+    cfg = inputs.PREFILL_CONFIGS[args.workload]
+    case = inputs.make_prefill_case(cfg, seed=rank_seed(cfg, rank))
+    step = PrefillStep(case, device)
+    flops = case.flops()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t_start.elapsed_time(t_stop)
+
+    # roofline pass: the attention launch bracketed by events on its stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        step.write()
+        ev[i][0].record(stream)
+        step.attend()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    att_ms = [a.elapsed_time(b) for a, b in ev]
+
+    soak_until = wall0 + 2.5
+    while time.time() < soak_until:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
+    wall_soak = time.time()
+    sampler.stop()
+
+    e2e = run_e2e_prefill(step, args.steps, args.warmup)
+    max_ms = all_reduce_max(elapsed_ms, world, device)
+    total_flops = all_reduce_sum(float(flops), world, device)
+    e2e_ms = all_reduce_max(e2e["ms"], world, device)
+    if rank != 0:
+        return None
+    value = total_flops * args.steps / (max_ms * 1e-3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+    att_avg = statistics.mean(att_ms)
+    achieved = flops / (att_avg * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.dtype,
+        "data": "synthetic (seeded N(0,1) Q/K/V, shuffled block pool)",
+        "config": {
+            "workload": cfg.name,
+            "description": cfg.description,
+            "num_seqs_per_gpu": case.cfg.num_seqs,
+            "num_heads": cfg.num_heads,
+            "num_kv_heads": cfg.num_kv_heads,
+            "head_dim": cfg.head_dim,
+            "block_size": cfg.block_size,
+            "query_tokens_per_step": case.num_tokens,
+            "context_lens": case.context_lens.tolist(),
+            "flops_per_step_per_gpu": flops,
+            "flops_rule": "4 * Hq * D per causally visible (query, key) pair (QK^T and PV multiply-adds)",
+            "step": "pa_reshape_and_cache (chunk K/V) + pa_prefill",
+            "l2": "inputs larger than L2: q, out, chunk K/V and the attended KV of a step total "
+                  f"{(2 * step.q.numel() * 2 + 2 * step.key.numel() * 2 + case.kv_bytes_attended()) / 2**20:.0f} MiB "
+                  "vs 126 MiB L2, no flush",
+            "parallelism": f"replicas x{world}, no data-path collective",
+        },
+        "pct_tensor_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {
+            "kernel": "pa_prefill",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_kind": "measured dense bf16 burst (MEASURED_PEAKS.json bf16_tflops)" if peak_kind == "measured"
+            else "fallback 1.59 PFLOP/s",
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": profiled_traffic(args.workload, kernel="pa_prefill"),
+            "prefill_ms_mean": round(att_avg, 5),
+            "prefill_ms_median": round(statistics.median(att_ms), 5),
+        },
+        "e2e": {"value": round(total_flops * args.steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": sampler.summary(wall0, wall_soak),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(case, budget_s=args.cpu_budget)
+    return line
+
+
+def run_e2e_prefill(step: PrefillStep, steps, warmup):
+    """Per step: q, the chunk K/V rows, slots and tables host->device from pinned
+    memory, the step through the public API, out device->host."""
+    case = step.case
+    pairs = [(step.q, case.q), (step.key, step.key_host), (step.value, step.value_host), (step.slots, step.slots_host),
+             (step.bt, case.block_tables), (step.cl, case.context_lens), (step.qsl, case.query_start_loc)]
+    pairs = [(d, h.pin_memory()) for d, h in pairs]
+    out_host = torch.empty(case.q.shape, dtype=case.q.dtype).pin_memory()
+    h2d = sum(h.numel() * h.element_size() for _, h in pairs)
+    d2h = out_host.numel() * out_host.element_size()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for d, h in pairs:
+            d.copy_(h, non_blocking=True)
+        step()
+        out_host.copy_(step.out, non_blocking=True)
+
+    for _ in range(max(1, warmup)):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return {"ms": a.elapsed_time(b), "h2d": h2d, "d2h": d2h}
+
+
+def _oracle_prefill(o, case):
+    return o.paged_prefill(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                           case.query_start_loc, case.scale)
+
+
+def _prefill_sample(case, budget_s):
+    """A bounded sample: the first sequences whose oracle run fits the budget (calibrated on one)."""
+    import oracle
+    o = oracle.get()
+    one = inputs.prefill_subcase(case, [0])
+    t = time.perf_counter()
+    _oracle_prefill(o, one)
+    per_flop = (time.perf_counter() - t) / max(1, one.flops())
+    n, fl = 0, 0
+    while n < case.cfg.num_seqs:
+        f = inputs.prefill_subcase(case, [n]).flops()
+        if n > 0 and (fl + f) * per_flop > budget_s:
+            break
+        fl += f
+        n += 1
+    return o, inputs.prefill_subcase(case, list(range(n))), n
+
+
+def cpu_baseline_prefill(case, budget_s: float = 20.0):
+    o, sample, n = _prefill_sample(case, budget_s / 2)
+    t = time.perf_counter()
+    _oracle_prefill(o, sample)
+    dt = time.perf_counter() - t
+    return {"value": round(sample.flops() / dt / 1e12, 6), "unit": "TFLOP/s", "cores": o.num_threads,
+            "kind": "oracle",
+            "sample": f"first {n} of {case.cfg.num_seqs} sequences of the same workload (whole chunks), fp64, one run"}
+
+
+def run_reference_prefill(args, world, rank):
+    if rank != 0:
+        return None
+    cfg = inputs.PREFILL_CONFIGS[args.workload]
+    case = inputs.make_prefill_case(cfg, seed=rank_seed(cfg, 0))
+    o, sample, n = _prefill_sample(case, args.ref_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _oracle_prefill(o, sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_prefill(o, sample)
+    el = time.perf_counter() - t0
+    value = sample.flops() * args.steps / el / 1e12
+    desc = f"first {n} of {cfg.num_seqs} sequences per step (fp64 paged prefill), {o.num_threads} threads"
+    return {
+        "metric": PREFILL_METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "description": cfg.description, "sample_seqs_per_step": n},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": o.num_threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
 def run_e2e(case, step, steps, warmup, device):
     """Per step: inputs host->device from pinned memory, the step through the
     public API, the output device->host into pinned memory."""
@@ -539,7 +802,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(inputs.CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=list(inputs.CONFIGS) + list(inputs.PREFILL_CONFIGS))
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds for the CPU-baseline sample")
     ap.add_argument("--ref-budget", type=float, default=120.0, help="seconds for the whole reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -548,10 +812,11 @@ def main(argv=None):
         ap.error("at least 3 warm-up steps")
     world, rank, local = dist_setup()
     try:
+        prefill = args.workload in inputs.PREFILL_CONFIGS
         if args.impl == "reference":
-            line = run_reference(args, world, rank)
+            line = (run_reference_prefill if prefill else run_reference)(args, world, rank)
         else:
-            line = run_ours(args, world, rank, local)
+            line = (run_prefill if prefill else run_ours)(args, world, rank, local)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

@@ -18,24 +18,34 @@
 // (row = query * G + head), so every K/V tile read from the cache serves all
 // grouped heads, and the two query tiles of a CTA share every K/V tile.  The
 // KV walk runs over tiles of 64 tokens (four cache blocks) up to the last
-// query's position.  Warp roles (320 threads):
+// query's position.  Warp roles (384 threads):
 //   warps 0-3, 4-7  one softmax warpgroup per query tile; thread = row.  Per KV
 //                   tile: tcgen05.ld of its 64 scores, causal mask on diagonal
 //                   tiles, online max/sum in base 2 (O rescaled in tensor
-//                   memory only when a row's max grows by more than 2^8), P to
-//                   shared memory as two 16-bit parts hi + lo (P carries ~16
-//                   bits, the accuracy of the decode kernel);
-//   warp 8          tensor-core issue: S = Q K^T (M=128 N=64, 8 x K=16) into a
-//                   double-buffered S, then O += P_hi V + P_lo V (M=128 N=128,
-//                   2 x 4 x K=16) for each query tile; the QK^T of tile j is
-//                   issued before the PV of tile j-1, so the tensor cores work
-//                   on one tile while the softmax runs on the previous one;
+//                   memory only when a row's max grows by more than 2^8), P
+//                   written back over its scores in tensor memory as two
+//                   16-bit parts hi + lo (P carries ~16 bits, the accuracy of
+//                   the decode kernel);
+//   warp 8          tensor-core issue: S = Q K^T (M=128 N=64, 8 x K=16, both
+//                   operands in shared memory) into a double-buffered S, and
+//                   O += P_hi V + P_lo V (M=128 N=128, 2 x 4 x K=16, P read
+//                   from tensor memory, V from shared memory), in the order
+//                   QK_A(j+1) PV_A(j) QK_B(j+1) PV_B(j): the tensor cores work
+//                   on one query tile while the softmax runs on the other;
 //   warp 9          TMA: K and V tiles (four 2 KiB boxes per 128-byte half of
 //                   the rows, 128-byte swizzled) into rings of 3 stages each,
-//                   block ids read from the block table one per lane.
-// Roles hand over through mbarriers only; every wait is bounded, and a role
-// that gives up raises a CTA-wide abort so that the others stop waiting.
-// Tensor memory: per query tile, S[2] (2 x 64 columns) and O (128 columns).
+//                   block ids read from the block table one per lane;
+//   warps 10-11     idle.
+// Roles hand over through mbarriers (one arrival per warp) only; every wait is
+// bounded, and a role that gives up raises a CTA-wide abort so that the others
+// stop waiting.  Each barrier is waited on by parity, so no barrier may complete
+// a phase twice before its waiter has seen the first: S and P hand-overs are
+// double-buffered by tile parity (writing P(j+2) needs S(j+2), issued only
+// after PV(j) has taken P(j)), and so is the PV-done hand-over (a waiter on
+// PV(j) has seen S(j+1), which needed PV(j-2) done); the K/V ring barriers
+// advance one phase per hand-over that their waiter itself enables.
+// Tensor memory: per query tile, S[2] (2 x 64 columns; P of a tile replaces
+// its S: 32 columns of hi pairs, then 32 of lo pairs) and O (128 columns).
 #pragma once
 
 #include "pa_common.cuh"
@@ -58,24 +68,24 @@ constexpr int kPrefillRows = 128;        // M: rows of one query tile
 constexpr int kPrefillTiles = 2;         // query tiles (softmax warpgroups) per CTA
 constexpr int kPrefillMmaWarp = 4 * kPrefillTiles;
 constexpr int kPrefillLoadWarp = kPrefillMmaWarp + 1;
-constexpr int kPrefillThreads = 32 * (kPrefillLoadWarp + 1);
+// three whole warpgroups: warps 10-11 only join the CTA barriers (ptxas fits
+// the softmax in the 168 registers of a 384-thread block without spilling)
+constexpr int kPrefillThreads = 128 * (kPrefillTiles + 1);
 constexpr int kPrefillKv = 64;           // N of S = Q K^T: tokens per KV tile
 constexpr int kPrefillKStages = 3;
 constexpr int kPrefillVStages = 3;
-constexpr int kPrefillTmemCols = 512;    // per query tile: S double buffer (2 x 64) + O (128)
+constexpr int kPrefillTmemCols = 512;    // per query tile: S/P double buffer (2 x 64) + O (128)
 constexpr float kRescaleLog2 = 8.f;      // rescale O once a row's max grows by more than this (base-2 units)
 
 struct PrefillSmem {
   static constexpr int kQTileBytes = 2 * kPrefillRows * 128;  // [2 halves][128 rows][128 B]
   static constexpr int kKvTileBytes = 2 * kPrefillKv * 128;   // [2 halves][64 tokens][128 B]
   static constexpr int kHalfBytes = kPrefillKv * 128;
-  static constexpr int kPBytes = kPrefillRows * 128;          // one part of P: [128 rows][64 tokens x 2 B]
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kPrefillTiles * kQTileBytes;
   static constexpr int kV = kK + kPrefillKStages * kKvTileBytes;
-  static constexpr int kP = kV + kPrefillVStages * kKvTileBytes;   // per query tile: P hi, then P lo
-  static constexpr int kBar = kP + kPrefillTiles * 2 * kPBytes;
-  // k_full[KS] v_full[VS] k_free[KS] v_free[VS]; per query tile: s_full[2] s_free[2] p_full o_done; drain
+  static constexpr int kBar = kV + kPrefillVStages * kKvTileBytes;
+  // k_full[KS] v_full[VS] k_free[KS] v_free[VS]; per query tile: s_full[2] p_full[2] o_done[2]; drain
   static constexpr int kTileBars = 6;
   static constexpr int kNumBars = 2 * (kPrefillKStages + kPrefillVStages) + kPrefillTiles * kTileBars + 1;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
@@ -92,11 +102,12 @@ struct Pack16<__nv_bfloat16> {
   static constexpr int kFormat = 1;   // tcgen05 kind::f16 operand format
   // p = hi + lo with hi = p truncated to bf16 (exact: the top 16 bits of p)
   // and lo = round(p - hi); two values per 32-bit word, a in the low half.
-  __device__ __forceinline__ static void split(float a, float b, uint32_t &hi, uint32_t &lo) {
-    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+  __device__ __forceinline__ static void split(float2 e, uint32_t &hi, uint32_t &lo) {
+    const uint32_t ua = __float_as_uint(e.x), ub = __float_as_uint(e.y);
     hi = __byte_perm(ua, ub, 0x7632);
-    __nv_bfloat162 l = __floats2bfloat162_rn(a - __uint_as_float(ua & 0xffff0000u),
-                                             b - __uint_as_float(ub & 0xffff0000u));
+    const float2 r = __ffma2_rn(make_float2(__uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u)),
+                                make_float2(-1.f, -1.f), e);   // e - hi, exact
+    __nv_bfloat162 l = __floats2bfloat162_rn(r.x, r.y);
     lo = *reinterpret_cast<uint32_t *>(&l);
   }
   __device__ __forceinline__ static uint32_t pack(float a, float b) {
@@ -107,10 +118,10 @@ struct Pack16<__nv_bfloat16> {
 template <>
 struct Pack16<__half> {
   static constexpr int kFormat = 0;
-  __device__ __forceinline__ static void split(float a, float b, uint32_t &hi, uint32_t &lo) {
-    const __half2 h = __floats2half2_rn(a, b);
+  __device__ __forceinline__ static void split(float2 e, uint32_t &hi, uint32_t &lo) {
+    const __half2 h = __floats2half2_rn(e.x, e.y);
     const float2 hf = __half22float2(h);
-    const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+    const __half2 l = __floats2half2_rn(e.x - hf.x, e.y - hf.y);
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
   }
@@ -145,10 +156,14 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
 }
 
 // Bounded wait that also gives up once another role has raised the abort flag.
-__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, const volatile int *abort_flag) {
+// With `backoff` the waiting warp sleeps between polls, leaving the shared
+// memory ports (which also feed the tensor cores' operands) to others.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, const volatile int *abort_flag,
+                                                   bool backoff = false) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
+    if (backoff) __nanosleep(64);
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0 && (*abort_flag || global_ns() - t0 > kWaitLimitNs)) return false;
   }
@@ -173,7 +188,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t *v_full = k_full + KS;
   uint64_t *k_free = v_full + VS;
   uint64_t *v_free = k_free + KS;
-  uint64_t *tile_bars = v_free + VS;   // query tile w: s_full[2], s_free[2], p_full, o_done at w * kTileBars
+  uint64_t *tile_bars = v_free + VS;   // query tile w: s_full[2], p_full[2], o_done[2] at w * kTileBars
   uint64_t *drain = tile_bars + NT * SM::kTileBars;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM::kTmemSlot);
   volatile int *abort_s = reinterpret_cast<int *>(smem + SM::kFlag);
@@ -226,10 +241,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint64_t *tb = tile_bars + w * SM::kTileBars;
       mbar_init(&tb[0], 1);               // s_full[0], s_full[1]: tensor-core commit
       mbar_init(&tb[1], 1);
-      mbar_init(&tb[2], kPrefillRows);    // s_free[0], s_free[1]: every softmax thread
-      mbar_init(&tb[3], kPrefillRows);
-      mbar_init(&tb[4], kPrefillRows);    // p_full: every softmax thread
-      mbar_init(&tb[5], 1);               // o_done: tensor-core commit
+      mbar_init(&tb[2], 4);               // p_full[0], p_full[1]: every softmax warp
+      mbar_init(&tb[3], 4);
+      mbar_init(&tb[4], 1);               // o_done[0], o_done[1]: tensor-core commit
+      mbar_init(&tb[5], 1);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -240,29 +255,42 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tmem_relinquish();
   }
 
-  // ---- Q tiles -> shared memory, K-major 128-byte swizzled: [d half][row][128 B]
+  tc_fence_before();
+  __syncthreads();   // barriers initialised, tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- Q tiles -> shared memory, K-major 128-byte swizzled: [d half][row][128 B].
+  // The TMA warp streams K/V meanwhile; only the tensor-core warp waits for Q
+  // (named barrier 1: the softmax warpgroups and the tensor-core warp).
   if (warp < kPrefillMmaWarp) {
     const int w = warp >> 2;
     const int q0 = (ct * NT + w) * QT;
     const int nq = max(0, min(QT, n - q0));
     const T *qg = reinterpret_cast<const T *>(p.q);
     uint8_t *q_s = smem + SM::kQ + w * SM::kQTileBytes;
-    for (int idx = tid & 127; idx < kPrefillRows * 16; idx += 128) {
-      const int row = idx >> 4, c = idx & 15;
+    const int c = tid & 15;              // this thread's 16-byte chunk of every row it moves
+    const int row0 = (tid & 127) >> 4;   // rows row0, row0 + 8, ...
+    uint4 x[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {   // every load in flight before the first store
+      const int row = row0 + 8 * k;
       const int i = row / G, hl = row % G;
-      uint4 x = make_uint4(0u, 0u, 0u, 0u);
+      x[k] = make_uint4(0u, 0u, 0u, 0u);
       if (i < nq)
-        x = *reinterpret_cast<const uint4 *>(
+        x[k] = *reinterpret_cast<const uint4 *>(
             qg + (static_cast<size_t>(qs + q0 + i) * p.num_heads + g * G + hl) * D + c * 8);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int row = row0 + 8 * k;
       *reinterpret_cast<uint4 *>(q_s + (c >> 3) * (kPrefillRows * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
-          x;
+          x[k];
     }
     fence_proxy_async_smem();   // the generic stores of Q are read by the tensor cores
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  if (warp <= kPrefillMmaWarp)
+    asm volatile("bar.sync 1, %0;" ::"n"(128 * kPrefillTiles + 32) : "memory");
 
   int last_k[KS], last_v[VS];   // TMA warp: last tile issued into each stage (for the abort drain)
 #pragma unroll
@@ -304,9 +332,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       else last_k[j % KS] = j;
     };
     for (int j = 0; j < ntiles; ++j) {
-      if (j >= KS && !__all_sync(kFullMask, mbar_wait_or_abort(&k_free[j % KS], (j / KS - 1) & 1, abort_s))) break;
+      if (j >= KS && !__all_sync(kFullMask, mbar_wait_or_abort(&k_free[j % KS], (j / KS - 1) & 1, abort_s, true))) break;
       issue(j, false);
-      if (j >= VS && !__all_sync(kFullMask, mbar_wait_or_abort(&v_free[j % VS], (j / VS - 1) & 1, abort_s))) break;
+      if (j >= VS && !__all_sync(kFullMask, mbar_wait_or_abort(&v_free[j % VS], (j / VS - 1) & 1, abort_s, true))) break;
       issue(j, true);
     }
   } else if (warp == kPrefillMmaWarp) {
@@ -324,74 +352,101 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tc_fence_after();
     };
     const bool zero_tail = (L & (kBlockSize - 1)) != 0 && (L - 1) / kBlockSize == pos_last_all / kBlockSize;
-    for (int j = 0; j <= ntiles && ok; ++j) {
-      if (j < ntiles) {
-        // ---- S_w(j) = Q_w K_j^T for every query tile that reaches KV tile j
-        wait(&k_full[j % KS], (j / KS) & 1);
-        const uint8_t *kt = smem + SM::kK + (j % KS) * SM::kKvTileBytes;
-        for (int w = 0; w < NT && ok; ++w) {
-          if (j >= nt[w]) continue;
-          uint64_t *tb = tile_bars + w * SM::kTileBars;
-          if (j >= 2) wait(&tb[2 + (j & 1)], ((j >> 1) - 1) & 1);   // S buffer j&1 read out (tile j-2)
-          if (!ok) break;
-          if (lane == 0) {
-            const uint8_t *q_s = smem + SM::kQ + w * SM::kQTileBytes;
-            const uint32_t d_tmem = tmem + w * 256 + (j & 1) * kPrefillKv;
+    // Issue order per KV tile j, query tile after query tile: QK_A(j+1), PV_A(j),
+    // QK_B(j+1), PV_B(j).  Every wait below is on work queued at least two
+    // groups earlier, so the tensor pipe does not drain at a hand-over, and
+    // each softmax warpgroup works while the other's products run.
+    //   S_w(j) = Q_w K_j^T goes to the S/P buffer j & 1 of query tile w, which
+    //   last held P_w(j-2); PV_w(j-2) reads that as its A operand straight from
+    //   tensor memory, and issue order does not keep a later product from
+    //   overwriting it, so QK_w(j) waits until PV_w(j-2) has completed.
+    // Descriptors are built once: an operand at byte offset `off` from a tile's
+    // base has the base's descriptor with off / 16 added to the start-address
+    // field (the field does not overflow: shared memory ends below 2^18 bytes).
+    // The issuing thread shares its scheduler with two softmax warps, so each
+    // product costs it as few instructions as possible.
+    const uint64_t q_desc = smem_desc_sw128(smem + SM::kQ, 16, 1024);
+    const uint64_t k_desc = smem_desc_sw128(smem + SM::kK, 16, 1024);
+    const uint64_t v_desc = smem_desc_sw128(smem + SM::kV, SM::kHalfBytes, 1024);
+    auto issue_qk = [&](int w, int j) {
+      uint64_t *tb = tile_bars + w * SM::kTileBars;
+      if (j >= 2) wait(&tb[4 + (j & 1)], ((j - 2) >> 1) & 1);   // PV_w(j-2) complete: buffer j&1 free
+      if (!ok) return;
+      if (lane == 0) {
+        const uint64_t a0 = q_desc + ((w * SM::kQTileBytes) >> 4);
+        const uint64_t b0 = k_desc + (((j % KS) * SM::kKvTileBytes) >> 4);
+        const uint32_t d_tmem = tmem + w * 256 + (j & 1) * kPrefillKv;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t a = smem_desc_sw128(q_s + (kk >> 2) * (kPrefillRows * 128) + (kk & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(kt + (kk >> 2) * SM::kHalfBytes + (kk & 3) * 32, 16, 1024);
-              umma_f16(d_tmem, a, bd, kIdescQK, kk > 0);
-            }
-            umma_commit(&tb[j & 1]);
-          }
-          __syncwarp();
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_f16(d_tmem, a0 + (((kk >> 2) * (kPrefillRows * 128) + (kk & 3) * 32) >> 4),
+                   b0 + (((kk >> 2) * SM::kHalfBytes + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
+        umma_commit(&tb[j & 1]);   // s_full
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int w, int j) {   // O_w += P_w(j) V_j
+      uint64_t *tb = tile_bars + w * SM::kTileBars;
+      wait(&tb[2 + (j & 1)], (j >> 1) & 1);   // P_w(j) written
+      if (!ok) return;
+      if (lane == 0) {
+        const uint64_t b0 = v_desc + (((j % VS) * SM::kKvTileBytes) >> 4);
+        const uint32_t a0 = tmem + w * 256 + (j & 1) * kPrefillKv;   // P_w(j): hi pairs, then lo pairs
+        const uint32_t o_tmem = tmem + w * 256 + 128;
+        const bool acc = j > 0;
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < kPrefillKv / 16; ++kk)   // 16 tokens = 8 columns of P per step
+            umma_f16_ts(o_tmem, a0 + part * 32 + kk * 8, b0 + ((kk * 16 * 128) >> 4), kIdescPV,
+                        acc || part > 0 || kk > 0);
+        umma_commit(&tb[4 + (j & 1)]);   // o_done
+      }
+      __syncwarp();
+    };
+    auto k_ready = [&](int j) { wait(&k_full[j % KS], (j / KS) & 1); };
+    auto v_ready = [&](int j) {
+      wait(&v_full[j % VS], (j / VS) & 1);
+      if (ok && zero_tail && j == ntiles - 1) {
+        // rows past the context end in its last block may hold anything (NaN
+        // included); make them zero so that 0 * V stays 0
+        uint8_t *vt = smem + SM::kV + (j % VS) * SM::kKvTileBytes;
+        const int t0 = j * kPrefillKv;
+        const int r0 = L - t0, r1 = ((L + kBlockSize - 1) / kBlockSize) * kBlockSize - t0;
+        for (int idx = lane; idx < (r1 - r0) * 16; idx += 32) {
+          const int r = r0 + (idx >> 4), c = idx & 15;
+          *reinterpret_cast<uint4 *>(vt + (c >> 3) * SM::kHalfBytes + r * 128 + (c & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
         }
-        if (ok && lane == 0) umma_commit(&k_free[j % KS]);   // K stage free once these products are done
+        fence_proxy_async_smem();
         __syncwarp();
       }
-      if (j >= 1 && ok) {
-        // ---- O_w += P_w(j-1) V_{j-1}
-        const int jv = j - 1;
-        wait(&v_full[jv % VS], (jv / VS) & 1);
-        if (!ok) break;
-        uint8_t *vt = smem + SM::kV + (jv % VS) * SM::kKvTileBytes;
-        if (zero_tail && jv == ntiles - 1) {
-          // rows past the context end in its last block may hold anything (NaN
-          // included); make them zero so that 0 * V stays 0
-          const int t0 = jv * kPrefillKv;
-          const int r0 = L - t0, r1 = ((L + kBlockSize - 1) / kBlockSize) * kBlockSize - t0;
-          for (int idx = lane; idx < (r1 - r0) * 16; idx += 32) {
-            const int r = r0 + (idx >> 4), c = idx & 15;
-            *reinterpret_cast<uint4 *>(vt + (c >> 3) * SM::kHalfBytes + r * 128 + (c & 7) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
+    };
+    if (ntiles > 0) {
+      k_ready(0);
+      for (int w = 0; w < NT && ok; ++w)
+        if (nt[w] > 0) issue_qk(w, 0);
+      if (ok && lane == 0) umma_commit(&k_free[0]);
+      __syncwarp();
+    }
+    for (int j = 0; j < ntiles && ok; ++j) {
+      bool k_in = false, v_in = false;
+      for (int w = 0; w < NT && ok; ++w) {
+        if (j + 1 < nt[w]) {
+          if (!k_in) k_ready(j + 1);
+          k_in = true;
+          if (ok) issue_qk(w, j + 1);
         }
-        for (int w = 0; w < NT && ok; ++w) {
-          if (jv >= nt[w]) continue;
-          uint64_t *tb = tile_bars + w * SM::kTileBars;
-          wait(&tb[4], jv & 1);   // P_w(jv) written
-          if (!ok) break;
-          if (lane == 0) {
-            const uint8_t *p_s = smem + SM::kP + w * 2 * SM::kPBytes;
-            const uint32_t o_tmem = tmem + w * 256 + 128;
-#pragma unroll
-            for (int part = 0; part < 2; ++part)
-#pragma unroll
-              for (int kk = 0; kk < kPrefillKv / 16; ++kk) {
-                const uint64_t a = smem_desc_sw128(p_s + part * SM::kPBytes + kk * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(vt + kk * 16 * 128, SM::kHalfBytes, 1024);
-                umma_f16(o_tmem, a, bd, kIdescPV, jv > 0 || part > 0 || kk > 0);
-              }
-            umma_commit(&tb[5]);
-          }
-          __syncwarp();
+        if (j < nt[w] && ok) {
+          if (!v_in) v_ready(j);
+          v_in = true;
+          if (ok) issue_pv(w, j);
         }
-        if (ok && lane == 0) umma_commit(&v_free[jv % VS]);
-        __syncwarp();
       }
+      if (ok && lane == 0) {
+        if (k_in) umma_commit(&k_free[(j + 1) % KS]);   // K stage free once its products are done
+        umma_commit(&v_free[j % VS]);
+      }
+      __syncwarp();
     }
   } else {
     // ================================================================ softmax warpgroup w
@@ -401,7 +456,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t t_s = tmem + w * 256 + lane_base;
     const uint32_t t_o = t_s + 128;
     uint64_t *tb = tile_bars + w * SM::kTileBars;
-    uint8_t *p_row = smem + SM::kP + w * 2 * SM::kPBytes + r * 128;
     const int q0 = (ct * NT + w) * QT;
     const int nq = max(0, min(QT, n - q0));
     const int i_row = r / G;
@@ -415,7 +469,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     bool ok = true;
     auto wait = [&](uint64_t *bar, uint32_t parity) {
       if (!ok) return;
-      ok = __all_sync(kFullMask, mbar_wait_or_abort(bar, parity, abort_s));
+      ok = __all_sync(kFullMask, mbar_wait_or_abort(bar, parity, abort_s, true));
       if (!ok && lane == 0) {
         record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, blockIdx.x);
         *abort_s = 1;
@@ -427,8 +481,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (!ok) break;
       float s[64];
       tmem_ld64(t_s + (j & 1) * kPrefillKv, s);
-      tc_fence_before();
-      mbar_arrive(&tb[2 + (j & 1)]);   // S buffer free for the tile after next
       const int t0 = j * kPrefillKv;
       if (t0 + kPrefillKv - 1 > pos_first) {   // a diagonal tile: mask tokens after each row's position
 #pragma unroll
@@ -450,22 +502,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         m_run = tmax;
         l_run *= f;
       }
-      const float mc = m_run * c2;
+      const float2 nmc = make_float2(-m_run * c2, -m_run * c2);
+      const float2 cc2 = make_float2(c2, c2);
       uint32_t ph[32], pl[32];
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 sum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const float a = ex2(fmaf(s[2 * k], c2, -mc));
-        const float bb = ex2(fmaf(s[2 * k + 1], c2, -mc));
-        sum[k & 3] += a + bb;
-        PK::split(a, bb, ph[k], pl[k]);
+        const float2 x = __ffma2_rn(make_float2(s[2 * k], s[2 * k + 1]), cc2, nmc);
+        const float2 e = make_float2(ex2(x.x), ex2(x.y));
+        sum[k & 1] = __fadd2_rn(sum[k & 1], e);
+        PK::split(e, ph[k], pl[k]);
       }
-      l_run += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      l_run += (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
 
-      // -- PV(j-1) done: P and O are free
-      if (j > 0) wait(&tb[5], (j - 1) & 1);
-      if (!ok) break;
+      // -- P(j) over S(j) in tensor memory (S(j) is in registers now)
+      tmem_st32u(t_s + (j & 1) * kPrefillKv, ph);
+      tmem_st32u(t_s + (j & 1) * kPrefillKv + 32, pl);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      // -- a row whose max grew: O, complete up to tile j-1, rescaled before PV(j)
       if (__any_sync(kFullMask, need)) {
+        wait(&tb[4 + ((j - 1) & 1)], ((j - 1) >> 1) & 1);   // PV(j-1) done; need implies j > 0
+        if (!ok) break;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           float o[32];
@@ -475,21 +532,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st32(t_o + c, o);
         }
       }
-      const int sw = r & 7;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        *reinterpret_cast<uint4 *>(p_row + ((cc ^ sw) << 4)) =
-            make_uint4(ph[4 * cc], ph[4 * cc + 1], ph[4 * cc + 2], ph[4 * cc + 3]);
-        *reinterpret_cast<uint4 *>(p_row + SM::kPBytes + ((cc ^ sw) << 4)) =
-            make_uint4(pl[4 * cc], pl[4 * cc + 1], pl[4 * cc + 2], pl[4 * cc + 3]);
-      }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&tb[4]);   // P(j) written (and O rescaled)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tb[2 + (j & 1)]);   // P(j) written (and O rescaled)
     }
     if (ok && ntw > 0) {
       // -- epilogue: O / l -> out
-      wait(&tb[5], (ntw - 1) & 1);
+      wait(&tb[4 + ((ntw - 1) & 1)], ((ntw - 1) >> 1) & 1);   // the last PV (and so every PV) done
       if (ok) {
         const float inv = 1.f / l_run;
         T *orow = reinterpret_cast<T *>(p.out) +

@@ -376,6 +376,12 @@ class PrefillCase:
         q = self.query_start_loc
         return int((q[1:] - q[:-1]).max()) if len(q) > 1 else 0
 
+    def kv_bytes_attended(self) -> int:
+        """Bytes of the K and V rows the chunks attend to (every cached token of each sequence)."""
+        c = self.cfg
+        return int(self.context_lens.to(torch.int64).sum()) * c.num_kv_heads * 2 * c.head_dim * \
+            self.k_cache.element_size()
+
     def flops(self) -> int:
         """Multiply-add flops of S = QK^T and O = PV over the causally visible keys."""
         c = self.cfg
