@@ -35,7 +35,7 @@
 //   warp 9          TMA: K and V tiles (four 2 KiB boxes per 128-byte half of
 //                   the rows, 128-byte swizzled) into rings of 3 stages each,
 //                   block ids read from the block table one per lane;
-//   warps 10-11     idle.
+//   warps 10-11     idle (as are lanes 1-31 of warp 8).
 // Roles hand over through mbarriers (one arrival per warp) only; every wait is
 // bounded, and a role that gives up raises a CTA-wide abort so that the others
 // stop waiting.  Each barrier is waited on by parity, so no barrier may complete
@@ -153,6 +153,17 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Non-blocking: has phase `parity` of `bar` completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
 }
 
 // Bounded wait that also gives up once another role has raised the abort flag.
@@ -337,15 +348,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (j >= VS && !__all_sync(kFullMask, mbar_wait_or_abort(&v_free[j % VS], (j / VS - 1) & 1, abort_s, true))) break;
       issue(j, true);
     }
-  } else if (warp == kPrefillMmaWarp) {
+  } else if (warp == kPrefillMmaWarp && lane == 0) {
     // ================================================================ tensor-core issue
+    // One thread: the tensor pipe takes products about as fast as it runs them,
+    // so every cycle this thread spends elsewhere (waits, warp syncs) leaves it idle.
     constexpr uint32_t kIdescQK = instr_desc_f16(PK::kFormat, false, kPrefillRows, kPrefillKv);
     constexpr uint32_t kIdescPV = instr_desc_f16(PK::kFormat, true, kPrefillRows, D);
     bool ok = true;
     auto wait = [&](uint64_t *bar, uint32_t parity) {
       if (!ok) return;
-      ok = __all_sync(kFullMask, mbar_wait_or_abort(bar, parity, abort_s));
-      if (!ok && lane == 0) {
+      ok = mbar_test_wait(bar, parity) || mbar_wait_or_abort(bar, parity, abort_s);
+      if (!ok) {
         record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, blockIdx.x);
         *abort_s = 1;
       }
@@ -372,7 +385,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint64_t *tb = tile_bars + w * SM::kTileBars;
       if (j >= 2) wait(&tb[4 + (j & 1)], ((j - 2) >> 1) & 1);   // PV_w(j-2) complete: buffer j&1 free
       if (!ok) return;
-      if (lane == 0) {
+      {
         const uint64_t a0 = q_desc + ((w * SM::kQTileBytes) >> 4);
         const uint64_t b0 = k_desc + (((j % KS) * SM::kKvTileBytes) >> 4);
         const uint32_t d_tmem = tmem + w * 256 + (j & 1) * kPrefillKv;
@@ -382,13 +395,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                    b0 + (((kk >> 2) * SM::kHalfBytes + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
         umma_commit(&tb[j & 1]);   // s_full
       }
-      __syncwarp();
     };
     auto issue_pv = [&](int w, int j) {   // O_w += P_w(j) V_j
       uint64_t *tb = tile_bars + w * SM::kTileBars;
       wait(&tb[2 + (j & 1)], (j >> 1) & 1);   // P_w(j) written
       if (!ok) return;
-      if (lane == 0) {
+      {
         const uint64_t b0 = v_desc + (((j % VS) * SM::kKvTileBytes) >> 4);
         const uint32_t a0 = tmem + w * 256 + (j & 1) * kPrefillKv;   // P_w(j): hi pairs, then lo pairs
         const uint32_t o_tmem = tmem + w * 256 + 128;
@@ -401,7 +413,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         acc || part > 0 || kk > 0);
         umma_commit(&tb[4 + (j & 1)]);   // o_done
       }
-      __syncwarp();
     };
     auto k_ready = [&](int j) { wait(&k_full[j % KS], (j / KS) & 1); };
     auto v_ready = [&](int j) {
@@ -412,21 +423,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         uint8_t *vt = smem + SM::kV + (j % VS) * SM::kKvTileBytes;
         const int t0 = j * kPrefillKv;
         const int r0 = L - t0, r1 = ((L + kBlockSize - 1) / kBlockSize) * kBlockSize - t0;
-        for (int idx = lane; idx < (r1 - r0) * 16; idx += 32) {
+        for (int idx = 0; idx < (r1 - r0) * 16; ++idx) {
           const int r = r0 + (idx >> 4), c = idx & 15;
           *reinterpret_cast<uint4 *>(vt + (c >> 3) * SM::kHalfBytes + r * 128 + (c & 7) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
-        __syncwarp();
       }
     };
     if (ntiles > 0) {
       k_ready(0);
       for (int w = 0; w < NT && ok; ++w)
         if (nt[w] > 0) issue_qk(w, 0);
-      if (ok && lane == 0) umma_commit(&k_free[0]);
-      __syncwarp();
+      if (ok) umma_commit(&k_free[0]);
     }
     for (int j = 0; j < ntiles && ok; ++j) {
       bool k_in = false, v_in = false;
@@ -442,13 +451,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (ok) issue_pv(w, j);
         }
       }
-      if (ok && lane == 0) {
+      if (ok) {
         if (k_in) umma_commit(&k_free[(j + 1) % KS]);   // K stage free once its products are done
         umma_commit(&v_free[j % VS]);
       }
-      __syncwarp();
     }
-  } else {
+  } else if (warp < kPrefillMmaWarp) {
     // ================================================================ softmax warpgroup w
     const int w = warp >> 2;
     const int r = tid & 127;             // row = tensor-memory lane
@@ -561,21 +569,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tc_fence_before();
   }
 
-  // ---- all roles done.  After an abort, let the copies and tensor-core
-  // operations in flight finish (bounded) before the memory is released.
+  // ---- all roles done.  Every tensor-core operation, and every barrier arrival
+  // that a commit makes, lands before the memory is released; after an abort
+  // the copies in flight are let finish too (all bounded).
   __syncthreads();
-  if (*abort_s) {
-    if (warp == kPrefillLoadWarp && lane == 0) {
-      // every stage: the last tile issued into it (its earlier phases completed before it was reissued)
-      for (int i = 0; i < KS; ++i)
-        if (last_k[i] >= 0) mbar_wait(&k_full[i], (last_k[i] / KS) & 1);
-      for (int i = 0; i < VS; ++i)
-        if (last_v[i] >= 0) mbar_wait(&v_full[i], (last_v[i] / VS) & 1);
-    }
-    if (warp == kPrefillMmaWarp && lane == 0) {
-      umma_commit(drain);
-      mbar_wait(drain, 0);
-    }
+  if (warp == kPrefillMmaWarp && lane == 0) {
+    umma_commit(drain);
+    mbar_wait(drain, 0);
+  }
+  if (*abort_s && warp == kPrefillLoadWarp && lane == 0) {
+    // every stage: the last tile issued into it (its earlier phases completed before it was reissued)
+    for (int i = 0; i < KS; ++i)
+      if (last_k[i] >= 0) mbar_wait(&k_full[i], (last_k[i] / KS) & 1);
+    for (int i = 0; i < VS; ++i)
+      if (last_v[i] >= 0) mbar_wait(&v_full[i], (last_v[i] / VS) & 1);
   }
   __syncthreads();
   if (warp == kPrefillMmaWarp) {
