@@ -26,16 +26,16 @@
 //                   written back over its scores in tensor memory as two
 //                   16-bit parts hi + lo (P carries ~16 bits, the accuracy of
 //                   the decode kernel);
-//   warp 8          tensor-core issue: S = Q K^T (M=128 N=64, 8 x K=16, both
-//                   operands in shared memory) into a double-buffered S, and
-//                   O += P_hi V + P_lo V (M=128 N=128, 2 x 4 x K=16, P read
-//                   from tensor memory, V from shared memory), in the order
-//                   QK_A(j+1) PV_A(j) QK_B(j+1) PV_B(j): the tensor cores work
-//                   on one query tile while the softmax runs on the other;
+//   warps 8, 10     tensor-core issue, one thread per query tile: S = Q K^T
+//                   (M=128 N=64, 8 x K=16, both operands in shared memory)
+//                   into a double-buffered S, and O += P_hi V + P_lo V (M=128
+//                   N=128, 2 x 4 x K=16, P read from tensor memory, V from
+//                   shared memory), QK(j+1) before PV(j); the tensor pipe runs
+//                   one query tile's products while the other's issuer waits;
 //   warp 9          TMA: K and V tiles (four 2 KiB boxes per 128-byte half of
 //                   the rows, 128-byte swizzled) into rings of 3 stages each,
 //                   block ids read from the block table one per lane;
-//   warps 10-11     idle (as are lanes 1-31 of warp 8).
+//   warp 11         idle (as are lanes 1-31 of warps 8 and 10).
 // Roles hand over through mbarriers (one arrival per warp) only; every wait is
 // bounded, and a role that gives up raises a CTA-wide abort so that the others
 // stop waiting.  Each barrier is waited on by parity, so no barrier may complete
@@ -85,9 +85,9 @@ struct PrefillSmem {
   static constexpr int kK = kQ + kPrefillTiles * kQTileBytes;
   static constexpr int kV = kK + kPrefillKStages * kKvTileBytes;
   static constexpr int kBar = kV + kPrefillVStages * kKvTileBytes;
-  // k_full[KS] v_full[VS] k_free[KS] v_free[VS]; per query tile: s_full[2] p_full[2] o_done[2]; drain
+  // k_full[KS] v_full[VS] k_free[KS] v_free[VS]; per query tile: s_full[2] p_full[2] o_done[2]; drain, tail_ready
   static constexpr int kTileBars = 6;
-  static constexpr int kNumBars = 2 * (kPrefillKStages + kPrefillVStages) + kPrefillTiles * kTileBars + 1;
+  static constexpr int kNumBars = 2 * (kPrefillKStages + kPrefillVStages) + kPrefillTiles * kTileBars + 2;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
   static constexpr int kFlag = kTmemSlot + 4;
   static constexpr int kBytes = kFlag + 4;
@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t *v_free = k_free + KS;
   uint64_t *tile_bars = v_free + VS;   // query tile w: s_full[2], p_full[2], o_done[2] at w * kTileBars
   uint64_t *drain = tile_bars + NT * SM::kTileBars;
+  uint64_t *tail_ready = drain + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM::kTmemSlot);
   volatile int *abort_s = reinterpret_cast<int *>(smem + SM::kFlag);
 
@@ -242,11 +243,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefetch_tensor_map(&tm_v);
     for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_free[i], 1);
+      mbar_init(&k_free[i], NT);   // one arrival per issuing thread
     }
     for (int i = 0; i < VS; ++i) {
       mbar_init(&v_full[i], 1);
-      mbar_init(&v_free[i], 1);
+      mbar_init(&v_free[i], NT);
     }
     for (int w = 0; w < NT; ++w) {
       uint64_t *tb = tile_bars + w * SM::kTileBars;
@@ -257,7 +258,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(&tb[4], 1);               // o_done[0], o_done[1]: tensor-core commit
       mbar_init(&tb[5], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, NT);
+    mbar_init(tail_ready, 1);
     fence_mbar_init();
     *abort_s = 0;
   }
@@ -272,8 +274,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   // ---- Q tiles -> shared memory, K-major 128-byte swizzled: [d half][row][128 B].
-  // The TMA warp streams K/V meanwhile; only the tensor-core warp waits for Q
-  // (named barrier 1: the softmax warpgroups and the tensor-core warp).
+  // The TMA warp streams K/V meanwhile; only the issuing warps wait for Q
+  // (named barrier 1: the softmax warpgroups and warps 8 and 10).
   if (warp < kPrefillMmaWarp) {
     const int w = warp >> 2;
     const int q0 = (ct * NT + w) * QT;
@@ -300,8 +302,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     fence_proxy_async_smem();   // the generic stores of Q are read by the tensor cores
   }
-  if (warp <= kPrefillMmaWarp)
-    asm volatile("bar.sync 1, %0;" ::"n"(128 * kPrefillTiles + 32) : "memory");
+  if (warp < kPrefillMmaWarp || warp == kPrefillMmaWarp || warp == kPrefillMmaWarp + 2)
+    asm volatile("bar.sync 1, %0;" ::"n"(128 * kPrefillTiles + 64) : "memory");
 
   int last_k[KS], last_v[VS];   // TMA warp: last tile issued into each stage (for the abort drain)
 #pragma unroll
@@ -348,10 +350,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (j >= VS && !__all_sync(kFullMask, mbar_wait_or_abort(&v_free[j % VS], (j / VS - 1) & 1, abort_s, true))) break;
       issue(j, true);
     }
-  } else if (warp == kPrefillMmaWarp && lane == 0) {
+  } else if ((warp == kPrefillMmaWarp || warp == kPrefillMmaWarp + 2) && lane == 0) {
     // ================================================================ tensor-core issue
-    // One thread: the tensor pipe takes products about as fast as it runs them,
-    // so every cycle this thread spends elsewhere (waits, warp syncs) leaves it idle.
+    // One thread per query tile w (warps 8 and 10, on different schedulers).
+    // The tensor pipe takes products about as fast as it runs them, so while
+    // one issuer waits on a hand-over the other keeps the pipe busy.
+    const int w = warp == kPrefillMmaWarp ? 0 : 1;
+    const int ntw = nt[w];
+    uint64_t *tb = tile_bars + w * SM::kTileBars;
     constexpr uint32_t kIdescQK = instr_desc_f16(PK::kFormat, false, kPrefillRows, kPrefillKv);
     constexpr uint32_t kIdescPV = instr_desc_f16(PK::kFormat, true, kPrefillRows, D);
     bool ok = true;
@@ -364,11 +370,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       tc_fence_after();
     };
+    // the K or V stage of tile t: an issuer with no product on t still arrives
+    // once, after the stage's previous phase has completed (so that its
+    // arrival counts toward tile t's phase)
+    auto free_arrive = [&](uint64_t *ring, int t, int stages) {
+      if (t >= stages) wait(&ring[t % stages], (t / stages - 1) & 1);
+      if (ok) mbar_arrive(&ring[t % stages]);
+    };
     const bool zero_tail = (L & (kBlockSize - 1)) != 0 && (L - 1) / kBlockSize == pos_last_all / kBlockSize;
-    // Issue order per KV tile j, query tile after query tile: QK_A(j+1), PV_A(j),
-    // QK_B(j+1), PV_B(j).  Every wait below is on work queued at least two
-    // groups earlier, so the tensor pipe does not drain at a hand-over, and
-    // each softmax warpgroup works while the other's products run.
+    const int tail_owner = nt[NT - 1] > 0 ? NT - 1 : 0;   // a query tile that reaches the last KV tile
+    // Per KV tile j: QK_w(j+1), then PV_w(j), so that the scores of the next
+    // tile are computed while the softmax works on this one.
     //   S_w(j) = Q_w K_j^T goes to the S/P buffer j & 1 of query tile w, which
     //   last held P_w(j-2); PV_w(j-2) reads that as its A operand straight from
     //   tensor memory, and issue order does not keep a later product from
@@ -376,85 +388,69 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // Descriptors are built once: an operand at byte offset `off` from a tile's
     // base has the base's descriptor with off / 16 added to the start-address
     // field (the field does not overflow: shared memory ends below 2^18 bytes).
-    // The issuing thread shares its scheduler with two softmax warps, so each
-    // product costs it as few instructions as possible.
-    const uint64_t q_desc = smem_desc_sw128(smem + SM::kQ, 16, 1024);
+    const uint64_t a_qk = smem_desc_sw128(smem + SM::kQ + w * SM::kQTileBytes, 16, 1024);
     const uint64_t k_desc = smem_desc_sw128(smem + SM::kK, 16, 1024);
     const uint64_t v_desc = smem_desc_sw128(smem + SM::kV, SM::kHalfBytes, 1024);
-    auto issue_qk = [&](int w, int j) {
-      uint64_t *tb = tile_bars + w * SM::kTileBars;
+    auto issue_qk = [&](int j) {
+      wait(&k_full[j % KS], (j / KS) & 1);
       if (j >= 2) wait(&tb[4 + (j & 1)], ((j - 2) >> 1) & 1);   // PV_w(j-2) complete: buffer j&1 free
       if (!ok) return;
-      {
-        const uint64_t a0 = q_desc + ((w * SM::kQTileBytes) >> 4);
-        const uint64_t b0 = k_desc + (((j % KS) * SM::kKvTileBytes) >> 4);
-        const uint32_t d_tmem = tmem + w * 256 + (j & 1) * kPrefillKv;
+      const uint64_t b0 = k_desc + (((j % KS) * SM::kKvTileBytes) >> 4);
+      const uint32_t d_tmem = tmem + w * 256 + (j & 1) * kPrefillKv;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_f16(d_tmem, a0 + (((kk >> 2) * (kPrefillRows * 128) + (kk & 3) * 32) >> 4),
-                   b0 + (((kk >> 2) * SM::kHalfBytes + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
-        umma_commit(&tb[j & 1]);   // s_full
-      }
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_f16(d_tmem, a_qk + (((kk >> 2) * (kPrefillRows * 128) + (kk & 3) * 32) >> 4),
+                 b0 + (((kk >> 2) * SM::kHalfBytes + (kk & 3) * 32) >> 4), kIdescQK, kk > 0);
+      umma_commit(&tb[j & 1]);              // s_full
+      umma_commit(&k_free[j % KS]);         // this issuer is done with the K stage once they complete
     };
-    auto issue_pv = [&](int w, int j) {   // O_w += P_w(j) V_j
-      uint64_t *tb = tile_bars + w * SM::kTileBars;
+    auto issue_pv = [&](int j) {   // O_w += P_w(j) V_j
+      wait(&v_full[j % VS], (j / VS) & 1);
+      if (!ok) return;
+      uint8_t *vt = smem + SM::kV + (j % VS) * SM::kKvTileBytes;
+      if (zero_tail && j == ntiles - 1) {
+        if (w == tail_owner) {
+          // rows past the context end in its last block may hold anything (NaN
+          // included); make them zero so that 0 * V stays 0
+          const int t0 = j * kPrefillKv;
+          const int r0 = L - t0, r1 = ((L + kBlockSize - 1) / kBlockSize) * kBlockSize - t0;
+          for (int idx = 0; idx < (r1 - r0) * 16; ++idx) {
+            const int r = r0 + (idx >> 4), c = idx & 15;
+            *reinterpret_cast<uint4 *>(vt + (c >> 3) * SM::kHalfBytes + r * 128 + (c & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(tail_ready);
+        } else {
+          wait(tail_ready, 0);
+          if (!ok) return;
+        }
+      }
       wait(&tb[2 + (j & 1)], (j >> 1) & 1);   // P_w(j) written
       if (!ok) return;
-      {
-        const uint64_t b0 = v_desc + (((j % VS) * SM::kKvTileBytes) >> 4);
-        const uint32_t a0 = tmem + w * 256 + (j & 1) * kPrefillKv;   // P_w(j): hi pairs, then lo pairs
-        const uint32_t o_tmem = tmem + w * 256 + 128;
-        const bool acc = j > 0;
+      const uint64_t b0 = v_desc + (((j % VS) * SM::kKvTileBytes) >> 4);
+      const uint32_t a0 = tmem + w * 256 + (j & 1) * kPrefillKv;   // P_w(j): hi pairs, then lo pairs
+      const uint32_t o_tmem = tmem + w * 256 + 128;
+      const bool acc = j > 0;
 #pragma unroll
-        for (int part = 0; part < 2; ++part)
+      for (int part = 0; part < 2; ++part)
 #pragma unroll
-          for (int kk = 0; kk < kPrefillKv / 16; ++kk)   // 16 tokens = 8 columns of P per step
-            umma_f16_ts(o_tmem, a0 + part * 32 + kk * 8, b0 + ((kk * 16 * 128) >> 4), kIdescPV,
-                        acc || part > 0 || kk > 0);
-        umma_commit(&tb[4 + (j & 1)]);   // o_done
-      }
+        for (int kk = 0; kk < kPrefillKv / 16; ++kk)   // 16 tokens = 8 columns of P per step
+          umma_f16_ts(o_tmem, a0 + part * 32 + kk * 8, b0 + ((kk * 16 * 128) >> 4), kIdescPV,
+                      acc || part > 0 || kk > 0);
+      umma_commit(&tb[4 + (j & 1)]);   // o_done
+      umma_commit(&v_free[j % VS]);    // this issuer is done with the V stage once they complete
     };
-    auto k_ready = [&](int j) { wait(&k_full[j % KS], (j / KS) & 1); };
-    auto v_ready = [&](int j) {
-      wait(&v_full[j % VS], (j / VS) & 1);
-      if (ok && zero_tail && j == ntiles - 1) {
-        // rows past the context end in its last block may hold anything (NaN
-        // included); make them zero so that 0 * V stays 0
-        uint8_t *vt = smem + SM::kV + (j % VS) * SM::kKvTileBytes;
-        const int t0 = j * kPrefillKv;
-        const int r0 = L - t0, r1 = ((L + kBlockSize - 1) / kBlockSize) * kBlockSize - t0;
-        for (int idx = 0; idx < (r1 - r0) * 16; ++idx) {
-          const int r = r0 + (idx >> 4), c = idx & 15;
-          *reinterpret_cast<uint4 *>(vt + (c >> 3) * SM::kHalfBytes + r * 128 + (c & 7) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-      }
-    };
-    if (ntiles > 0) {
-      k_ready(0);
-      for (int w = 0; w < NT && ok; ++w)
-        if (nt[w] > 0) issue_qk(w, 0);
-      if (ok) umma_commit(&k_free[0]);
-    }
+    if (ntw > 0) issue_qk(0);
+    else free_arrive(k_free, 0, KS);
     for (int j = 0; j < ntiles && ok; ++j) {
-      bool k_in = false, v_in = false;
-      for (int w = 0; w < NT && ok; ++w) {
-        if (j + 1 < nt[w]) {
-          if (!k_in) k_ready(j + 1);
-          k_in = true;
-          if (ok) issue_qk(w, j + 1);
-        }
-        if (j < nt[w] && ok) {
-          if (!v_in) v_ready(j);
-          v_in = true;
-          if (ok) issue_pv(w, j);
-        }
+      if (j + 1 < ntiles) {
+        if (j + 1 < ntw) issue_qk(j + 1);
+        else free_arrive(k_free, j + 1, KS);
       }
-      if (ok) {
-        if (k_in) umma_commit(&k_free[(j + 1) % KS]);   // K stage free once its products are done
-        umma_commit(&v_free[j % VS]);
-      }
+      if (!ok) break;
+      if (j < ntw) issue_pv(j);
+      else free_arrive(v_free, j, VS);
     }
   } else if (warp < kPrefillMmaWarp) {
     // ================================================================ softmax warpgroup w
@@ -573,8 +569,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   // that a commit makes, lands before the memory is released; after an abort
   // the copies in flight are let finish too (all bounded).
   __syncthreads();
-  if (warp == kPrefillMmaWarp && lane == 0) {
-    umma_commit(drain);
+  if ((warp == kPrefillMmaWarp || warp == kPrefillMmaWarp + 2) && lane == 0) {
+    umma_commit(drain);   // both issuers: their own operations (and commit arrivals) complete
     mbar_wait(drain, 0);
   }
   if (*abort_s && warp == kPrefillLoadWarp && lane == 0) {
