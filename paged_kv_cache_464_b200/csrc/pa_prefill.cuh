@@ -24,8 +24,8 @@
 //                   tiles, online max/sum in base 2 (O rescaled in tensor
 //                   memory only when a row's max grows by more than 2^8), P
 //                   written back over its scores in tensor memory as two
-//                   16-bit parts hi + lo (P carries ~16 bits, the accuracy of
-//                   the decode kernel);
+//                   16-bit parts hi + lo (P carries ~15 bits or more, like the
+//                   decode kernel);
 //   warps 8, 10     tensor-core issue, one thread per query tile: S = Q K^T
 //                   (M=128 N=64, 8 x K=16, both operands in shared memory)
 //                   into a double-buffered S, and O += P_hi V + P_lo V (M=128
@@ -100,15 +100,16 @@ struct Pack16;
 template <>
 struct Pack16<__nv_bfloat16> {
   static constexpr int kFormat = 1;   // tcgen05 kind::f16 operand format
-  // p = hi + lo with hi = p truncated to bf16 (exact: the top 16 bits of p)
-  // and lo = round(p - hi); two values per 32-bit word, a in the low half.
+  // p = hi + lo + t: hi = the top 16 bits of p (p truncated to bf16), lo = the
+  // top 16 bits of the exact remainder p - hi; |t| < 2^-15 |p|.  Integer
+  // work only (no conversion instructions); two values per 32-bit word, the
+  // first in the low half.
   __device__ __forceinline__ static void split(float2 e, uint32_t &hi, uint32_t &lo) {
     const uint32_t ua = __float_as_uint(e.x), ub = __float_as_uint(e.y);
     hi = __byte_perm(ua, ub, 0x7632);
     const float2 r = __ffma2_rn(make_float2(__uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u)),
                                 make_float2(-1.f, -1.f), e);   // e - hi, exact
-    __nv_bfloat162 l = __floats2bfloat162_rn(r.x, r.y);
-    lo = *reinterpret_cast<uint32_t *>(&l);
+    lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
   }
   __device__ __forceinline__ static uint32_t pack(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
