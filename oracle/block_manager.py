@@ -51,18 +51,26 @@ class PagedBlockManager:
     def slots(self, seq: int, start: int, stop: int) -> List[int]:
         return [self._slot(seq, p) for p in range(start, stop)]
 
+    def _available(self) -> int:
+        """Blocks an allocation may take."""
+        return len(self.free_blocks)
+
+    def _take(self) -> int:
+        """The next block to hand out: the front of the free list."""
+        return self.free_blocks.pop(0)
+
     # -- allocate_request ------------------------------------------------------------
     def allocate(self, seq: int, num_tokens: int) -> List[int]:
         """Blocks for a new request's prompt: ceil(n / bs) blocks from the front of
         the free list, reference count 1.  Returns the slots of the n tokens."""
         assert seq not in self.block_tables
         need = math.ceil(num_tokens / self.block_size)
-        if need > len(self.free_blocks):
+        if need > self._available():
             raise NoSpace(seq)
         table = []
         left = num_tokens
         for _ in range(need):
-            b = self.free_blocks.pop(0)
+            b = self._take()
             self.ref_count[b] = 1
             self.num_tokens[b] = min(self.block_size, left)
             left -= self.num_tokens[b]
@@ -83,9 +91,9 @@ class PagedBlockManager:
         if table and offset != 0:
             last = table[-1]
             if self.ref_count[last] > 1:                        # shared: copy before writing
-                if not self.free_blocks:
+                if not self._available():
                     raise NoSpace(seq)
-                new = self.free_blocks.pop(0)
+                new = self._take()
                 self.ref_count[last] -= 1
                 self.ref_count[new] = 1
                 self.num_tokens[new] = offset
@@ -94,9 +102,9 @@ class PagedBlockManager:
                 last = new
             self.num_tokens[last] = offset + 1
         else:
-            if not self.free_blocks:
+            if not self._available():
                 raise NoSpace(seq)
-            last = self.free_blocks.pop(0)
+            last = self._take()
             self.ref_count[last] = 1
             self.num_tokens[last] = 1
             table.append(last)
@@ -129,14 +137,14 @@ class PagedBlockManager:
             else:
                 break
         need = math.ceil((num_tokens - covered) / self.block_size)
-        if need > len(self.free_blocks):
+        if need > self._available():
             raise NoSpace(seq)
         for b in shared:
             self.ref_count[b] += 1
         table = list(shared)
         left = num_tokens - covered
         for _ in range(need):
-            b = self.free_blocks.pop(0)
+            b = self._take()
             self.ref_count[b] = 1
             self.num_tokens[b] = min(self.block_size, left)
             left -= self.num_tokens[b]
