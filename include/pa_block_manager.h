@@ -15,6 +15,7 @@
  *       size 16 by default, copy-on-write: a request that writes into a shared
  *       block gets its own copy first.
  *   [C] "vLLM推理引擎深度实战：…" §1.2 -- running out of blocks is an error.
+ *   [B] "vLLM 原理与源码阅读", Prefix Caching -- see pa_bm_create_prefix_caching.
  *
  * Readings: the free list is first-in first-out (blocks are taken from its
  * front and returned to its back, as the pages' pop(0) / append do); a write
@@ -109,6 +110,53 @@ int32_t pa_bm_free_list(const pa_block_manager_t *bm, int32_t *out, int32_t cap)
 int32_t pa_bm_sequences(const pa_block_manager_t *bm, int64_t *out, int32_t cap);      /* count; ascending ids */
 int32_t pa_bm_table(const pa_block_manager_t *bm, int64_t seq, int32_t *out, int32_t cap); /* length or -1 */
 void pa_bm_stats(const pa_block_manager_t *bm, pa_bm_stats_t *out);
+
+/*
+ * Prefix caching ([B] Prefix Caching, 自动检测与复用: (1) a cache key from the
+ * prompt's content, (2) the longest cached prefix of a new request, (3) only
+ * the missed part computed, (4) the hit blocks shared by reference).
+ *
+ * Readings: the unit is a FULL prompt block (block_size tokens); a block's key
+ * is its token ids together with the cache entry of the block before it, so a
+ * hit on block i means the whole prefix up to block i is identical (keys are
+ * looked up by an FNV-1a hash and then compared exactly: a hash collision
+ * cannot share blocks).  Entry numbers are never reused.  Only prompt blocks
+ * are cached (decode tokens are not).  A cached block whose reference count
+ * drops to 0 keeps its content and becomes evictable; allocation takes the
+ * free list first and then evicts the least recently released cached block;
+ * a sequence releases its blocks last to first (pa_bm_free), so a cached
+ * block's prefix is always cached too.  Every other call of this header works
+ * on a prefix-caching manager as described above, taking evictable blocks
+ * when the free list is empty.
+ */
+typedef struct {
+  int64_t queried_blocks;    /* full prompt blocks looked up */
+  int64_t hit_blocks;        /* of those, found in the cache */
+  int64_t cached_blocks;     /* blocks currently in the cache (in use or evictable) */
+  int64_t evictable_blocks;  /* cached blocks with reference count 0 */
+  int64_t evictions;         /* cached blocks handed out for other content */
+} pa_bm_prefix_stats_t;
+
+/* A prefix-caching manager (otherwise as pa_bm_create). */
+pa_block_manager_t *pa_bm_create_prefix_caching(int32_t num_blocks, int32_t block_size);
+
+/* allocate_request with prefix caching: the longest run of leading full blocks
+ * of token_ids[num_tokens] found in the cache is shared (reference count + 1;
+ * an evictable block is taken back), new blocks hold the rest, and the new
+ * full blocks are cached.  slots (may be NULL) receives the slots of all
+ * num_tokens tokens; *num_cached_tokens (may be NULL) the number of leading
+ * tokens whose K/V are already in the cache (a multiple of block_size): the
+ * caller computes and writes only the tokens after them.  On a manager made by
+ * pa_bm_create it is pa_bm_allocate with *num_cached_tokens = 0. */
+pa_bm_status_t pa_bm_allocate_prompt(pa_block_manager_t *bm, int64_t seq, const int32_t *token_ids,
+                                     int32_t num_tokens, int64_t *slots, int32_t *num_cached_tokens);
+
+/* Inspection: the evictable blocks, oldest release first (count; first cap ids);
+ * whether a block is cached (1, with its entry and parent entry), not (0) or
+ * out of range (-1); counters. */
+int32_t pa_bm_evictable(const pa_block_manager_t *bm, int32_t *out, int32_t cap);
+int32_t pa_bm_cache_entry(const pa_block_manager_t *bm, int32_t block, int64_t *entry, int64_t *parent_entry);
+void pa_bm_prefix_stats(const pa_block_manager_t *bm, pa_bm_prefix_stats_t *out);
 
 #ifdef __cplusplus
 }

@@ -50,9 +50,28 @@ _lib.pa_bm_table.argtypes = [_P, _I64, _P, _I32]
 _lib.pa_bm_stats.restype = None
 _lib.pa_bm_stats.argtypes = [_P, ctypes.POINTER(_Stats)]
 
+
+class _PrefixStats(ctypes.Structure):
+    _fields_ = [("queried_blocks", ctypes.c_int64), ("hit_blocks", ctypes.c_int64),
+                ("cached_blocks", ctypes.c_int64), ("evictable_blocks", ctypes.c_int64),
+                ("evictions", ctypes.c_int64)]
+
+
+_lib.pa_bm_create_prefix_caching.restype = _P
+_lib.pa_bm_create_prefix_caching.argtypes = [_I32, _I32]
+_lib.pa_bm_allocate_prompt.restype = ctypes.c_int
+_lib.pa_bm_allocate_prompt.argtypes = [_P, _I64, _P, _I32, _P, ctypes.POINTER(_I32)]
+_lib.pa_bm_evictable.restype = _I32
+_lib.pa_bm_evictable.argtypes = [_P, _P, _I32]
+_lib.pa_bm_cache_entry.restype = _I32
+_lib.pa_bm_cache_entry.argtypes = [_P, _I32, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]
+_lib.pa_bm_prefix_stats.restype = None
+_lib.pa_bm_prefix_stats.argtypes = [_P, ctypes.POINTER(_PrefixStats)]
+
 EXPORTED = ["pa_bm_create", "pa_bm_destroy", "pa_bm_allocate", "pa_bm_share_prefix", "pa_bm_append",
             "pa_bm_append_batch", "pa_bm_free", "pa_bm_block_tables", "pa_bm_context_len", "pa_bm_ref_count",
-            "pa_bm_free_list", "pa_bm_sequences", "pa_bm_table", "pa_bm_stats"]
+            "pa_bm_free_list", "pa_bm_sequences", "pa_bm_table", "pa_bm_stats", "pa_bm_create_prefix_caching",
+            "pa_bm_allocate_prompt", "pa_bm_evictable", "pa_bm_cache_entry", "pa_bm_prefix_stats"]
 
 _STATUS = {0: "ok", 1: "no space", 2: "bad argument", 3: "unknown sequence", 4: "sequence exists",
            5: "table longer than max_blocks_per_seq"}
@@ -78,12 +97,14 @@ def _ptr(a: np.ndarray) -> int:
 
 
 class BlockManager:
-    """A pool of ``num_blocks`` KV blocks of ``block_size`` tokens."""
+    """A pool of ``num_blocks`` KV blocks of ``block_size`` tokens (with prefix
+    caching of full prompt blocks when ``prefix_caching``)."""
 
     NoSpace = NoSpace
 
-    def __init__(self, num_blocks: int, block_size: int = 16):
-        self._h = _lib.pa_bm_create(num_blocks, block_size)
+    def __init__(self, num_blocks: int, block_size: int = 16, prefix_caching: bool = False):
+        create = _lib.pa_bm_create_prefix_caching if prefix_caching else _lib.pa_bm_create
+        self._h = create(num_blocks, block_size)
         if not self._h:
             raise BlockManagerError("pa_bm_create failed")
         self.num_blocks = num_blocks
@@ -100,6 +121,16 @@ class BlockManager:
         slots = np.empty(max(num_tokens, 1), dtype=np.int64)
         _check(_lib.pa_bm_allocate(self._h, seq, num_tokens, _ptr(slots)), f"allocate({seq})")
         return slots[:num_tokens].tolist()
+
+    def allocate_prompt(self, seq: int, tokens: Sequence[int]) -> Tuple[List[int], int]:
+        """(slots of all prompt tokens, number of leading tokens already cached)."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = len(t)
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        cached = _I32(0)
+        _check(_lib.pa_bm_allocate_prompt(self._h, seq, _ptr(t) if n else None, n, _ptr(slots), ctypes.byref(cached)),
+               f"allocate_prompt({seq})")
+        return slots[:n].tolist(), cached.value
 
     def share_prefix(self, seq: int, src: int, num_tokens: int) -> List[int]:
         slots = np.empty(max(num_tokens, 1), dtype=np.int64)
@@ -185,3 +216,30 @@ class BlockManager:
     @property
     def ref_count(self) -> List[int]:
         return [int(_lib.pa_bm_ref_count(self._h, b)) for b in range(self.num_blocks)]
+
+    @property
+    def evictable(self) -> List[int]:
+        n = _lib.pa_bm_evictable(self._h, None, 0)
+        out = np.empty(max(n, 1), dtype=np.int32)
+        _lib.pa_bm_evictable(self._h, _ptr(out), n)
+        return out[:n].tolist()
+
+    def cache_items(self):
+        """(parent entry, None, block) of every cached block (token ids stay in the manager)."""
+        items = []
+        e, pe = _I64(0), _I64(0)
+        for b in range(self.num_blocks):
+            if _lib.pa_bm_cache_entry(self._h, b, ctypes.byref(e), ctypes.byref(pe)) == 1:
+                items.append((pe.value, None, b))
+        return items
+
+    def cache_entries(self) -> List[int]:
+        e, pe = _I64(0), _I64(0)
+        return [e.value for b in range(self.num_blocks)
+                if _lib.pa_bm_cache_entry(self._h, b, ctypes.byref(e), ctypes.byref(pe)) == 1]
+
+    def prefix_stats(self) -> Dict[str, int]:
+        st = _PrefixStats()
+        _lib.pa_bm_prefix_stats(self._h, ctypes.byref(st))
+        return {"queried_blocks": st.queried_blocks, "hit_blocks": st.hit_blocks, "cached_blocks": st.cached_blocks,
+                "evictable_blocks": st.evictable_blocks, "evictions": st.evictions}

@@ -15,7 +15,7 @@ def _prompt(rng: random.Random, prefix: List[int], extra: int) -> List[int]:
 
 
 def _table(m, seq):
-    return m.tables(seq) if hasattr(m, "tables") and callable(m.tables) else m.block_tables[seq]
+    return m.table(seq) if hasattr(m, "table") else m.block_tables[seq]
 
 
 def _check_state(m, live: Dict[int, List[int]], contents: Dict[int, List[int]]):
@@ -29,8 +29,9 @@ def _check_state(m, live: Dict[int, List[int]], contents: Dict[int, List[int]]):
             counts[b] += 1
             held = toks[i * bs:(i + 1) * bs]
             assert contents[b][:len(held)] == held, f"block {b} of seq {seq} holds other tokens"
+    rc = list(m.ref_count)
     for b in range(m.num_blocks):
-        assert m.ref_count[b] == counts[b], (b, m.ref_count[b], counts[b])
+        assert rc[b] == counts[b], (b, rc[b], counts[b])
     free, evictable = list(m.free_blocks), list(m.evictable)
     in_use = [b for b in range(m.num_blocks) if counts[b] > 0]
     assert sorted(free + evictable + in_use) == list(range(m.num_blocks)), "a block is lost or counted twice"
@@ -39,7 +40,8 @@ def _check_state(m, live: Dict[int, List[int]], contents: Dict[int, List[int]]):
 def _allocate(m, seq, toks, contents):
     """allocate_prompt plus the content model: new blocks receive the tokens they cover."""
     bs = m.block_size
-    before = set(b for b in range(m.num_blocks) if m.ref_count[b] > 0)
+    rc = list(m.ref_count)
+    before = set(b for b in range(m.num_blocks) if rc[b] > 0)
     slots, cached = m.allocate_prompt(seq, toks)
     t = _table(m, seq)
     assert cached % bs == 0 and cached <= len(toks)
@@ -56,7 +58,7 @@ def pin_longest_prefix_brute_force(cls):
     """Without evictions, the cached tokens of a prompt are the longest run of
     leading full blocks it shares with any earlier prompt still cached."""
     rng = random.Random(11)
-    m = cls(4096, 16)
+    m = cls(1024, 16)
     system = [rng.randrange(32000) for _ in range(70)]
     prompts: List[List[int]] = []
     contents: Dict[int, List[int]] = {}
