@@ -569,30 +569,9 @@ def run_e2e_prefill(step: PrefillStep, steps, warmup):
     """Per step: q, the chunk K/V rows, slots and tables host->device from pinned
     memory, the step through the public API, out device->host."""
     case = step.case
-    pairs = [(step.q, case.q), (step.key, step.key_host), (step.value, step.value_host), (step.slots, step.slots_host),
-             (step.bt, case.block_tables), (step.cl, case.context_lens), (step.qsl, case.query_start_loc)]
-    pairs = [(d, h.pin_memory()) for d, h in pairs]
-    out_host = torch.empty(case.q.shape, dtype=case.q.dtype).pin_memory()
-    h2d = sum(h.numel() * h.element_size() for _, h in pairs)
-    d2h = out_host.numel() * out_host.element_size()
-    stream = torch.cuda.current_stream()
-
-    def one():
-        for d, h in pairs:
-            d.copy_(h, non_blocking=True)
-        step()
-        out_host.copy_(step.out, non_blocking=True)
-
-    for _ in range(max(1, warmup)):
-        one()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
-    torch.cuda.synchronize()
-    return {"ms": a.elapsed_time(b), "h2d": h2d, "d2h": d2h}
+    host = {"q": case.q, "key": step.key_host, "value": step.value_host, "slots": step.slots_host,
+            "bt": case.block_tables, "cl": case.context_lens, "qsl": case.query_start_loc}
+    return pipelined_e2e(step, {k: t.pin_memory() for k, t in host.items()}, steps, warmup)
 
 
 def _oracle_prefill(o, case):
@@ -655,37 +634,77 @@ def run_reference_prefill(args, world, rank):
     }
 
 
+def pipelined_e2e(step, host, steps, warmup):
+    """End to end through the public API: every step copies its inputs `host`
+    (step attribute name -> pinned host tensor) to the device, runs `step()`
+    and copies `step.out` back into pinned host memory.  Two sets of device
+    inputs and outputs alternate between steps, with one copy stream per
+    direction, so that step k's copies overlap the kernels of step k-1 (as a
+    serving loop would run them); every copy of every timed step lies inside
+    the timed region."""
+    names = list(host)
+    compute = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    bufs = [{n: getattr(step, n) for n in names}, {n: torch.empty_like(getattr(step, n)) for n in names}]
+    outs = [step.out, torch.empty_like(step.out)]
+    out_host = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
+    loaded = [torch.cuda.Event() for _ in range(2)]     # inputs of set i on the device
+    consumed = [torch.cuda.Event() for _ in range(2)]   # kernels that read set i (and write its output) done
+    drained = [torch.cuda.Event() for _ in range(2)]    # output of set i copied to the host
+
+    def one(k):
+        i = k & 1
+        h2d_s.wait_event(consumed[i])                   # the step two back is done with these inputs
+        with torch.cuda.stream(h2d_s):
+            for n in names:
+                bufs[i][n].copy_(host[n], non_blocking=True)
+        loaded[i].record(h2d_s)
+        compute.wait_event(loaded[i])
+        compute.wait_event(drained[i])                  # its output buffer has been read out
+        for n in names:
+            setattr(step, n, bufs[i][n])
+        step.out = outs[i]
+        step()
+        consumed[i].record(compute)
+        d2h_s.wait_event(consumed[i])
+        with torch.cuda.stream(d2h_s):
+            out_host[i].copy_(outs[i], non_blocking=True)
+        drained[i].record(d2h_s)
+
+    def loop(n):
+        for i in range(2):
+            consumed[i].record(compute)
+            drained[i].record(compute)
+        h2d_s.wait_stream(compute)
+        d2h_s.wait_stream(compute)
+        for k in range(n):
+            one(k)
+        compute.wait_stream(h2d_s)
+        compute.wait_stream(d2h_s)
+
+    loop(max(2, warmup))
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(compute)
+    loop(steps)
+    b.record(compute)
+    torch.cuda.synchronize()
+    for n in names:
+        setattr(step, n, bufs[0][n])
+    step.out = outs[0]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    return {"ms": a.elapsed_time(b), "h2d": h2d, "d2h": d2h, "last_out_host": out_host[(steps - 1) & 1]}
+
+
 def run_e2e(case, step, steps, warmup, device):
     """Per step: inputs host->device from pinned memory, the step through the
     public API, the output device->host into pinned memory."""
-    pa = step.pa
-    host = {k: getattr(case, k).pin_memory() for k in ("q", "key", "value", "slot_mapping", "block_mapping",
-                                                         "block_tables", "context_lens")}
-    dev = {"q": step.q, "key": step.key, "value": step.value, "slot_mapping": step.slots,
-           "block_mapping": step.pairs, "block_tables": step.bt, "context_lens": step.cl}
-    out_host = torch.empty(case.q.shape, dtype=case.q.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for k, t in host.items() if k != "block_mapping" or step.has_pairs)
-    d2h = out_host.numel() * out_host.element_size()
-    stream = torch.cuda.current_stream()
-
-    def one():
-        for k, t in host.items():
-            if k == "block_mapping" and not step.has_pairs:
-                continue
-            dev[k].copy_(t, non_blocking=True)
-        step()
-        out_host.copy_(step.out, non_blocking=True)
-
-    for _ in range(max(1, warmup)):
-        one()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
-    torch.cuda.synchronize()
-    return {"ms": a.elapsed_time(b), "h2d": h2d, "d2h": d2h}
+    host = {"q": case.q, "key": case.key, "value": case.value, "slots": case.slot_mapping,
+            "bt": case.block_tables, "cl": case.context_lens}
+    if step.has_pairs:
+        host["pairs"] = case.block_mapping
+    return pipelined_e2e(step, {k: t.pin_memory() for k, t in host.items()}, steps, warmup)
 
 
 # ------------------------------------------------------------------ oracle timings
