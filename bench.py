@@ -92,6 +92,18 @@ def profiled_traffic(workload: str, kernel: str = "pa_decode"):
     return d.get("dram_bytes_per_call")
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi samples every 200 ms in a background process."""
@@ -603,7 +615,7 @@ def cpu_baseline_prefill(case, budget_s: float = 20.0):
     _oracle_prefill(o, sample)
     dt = time.perf_counter() - t
     return {"value": round(sample.flops() / dt / 1e12, 6), "unit": "TFLOP/s", "cores": o.num_threads,
-            "kind": "oracle",
+            "kind": "oracle", "cpu": cpu_model(),
             "sample": f"first {n} of {case.cfg.num_seqs} sequences of the same workload (whole chunks), fp64, one run"}
 
 
@@ -627,7 +639,7 @@ def run_reference_prefill(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": cfg.name, "description": cfg.description, "sample_seqs_per_step": n},
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": o.num_threads, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": o.num_threads, "kind": "oracle", "cpu": cpu_model(),
                          "sample": desc},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -770,10 +782,24 @@ def cpu_baseline(case, budget_s: float = 20.0):
         dt = time.perf_counter() - t
         best = dt if best is None else min(best, dt)
         reps += 1
-    return {"value": round(sample.kv_bytes() / best / 1e9, 4), "unit": "GB/s", "cores": o.num_threads,
-            "kind": "oracle", "seqs_per_s": round(n / best, 3),
+    # the same step on one thread, on a sample sized to a quarter of the budget
+    threads = o.num_threads
+    n1 = max(1, min(n, int(budget_s / 4 / max(per_seq * threads, 1e-6))))
+    sample1 = _sample_case(case, n1)
+    o.set_num_threads(1)
+    try:
+        t = time.perf_counter()
+        _oracle_step(o, sample1, k, v)
+        dt1 = time.perf_counter() - t
+    finally:
+        o.set_num_threads(threads)
+    return {"value": round(sample.kv_bytes() / best / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle", "cpu": cpu_model(), "seqs_per_s": round(n / best, 3),
             "sample": f"first {n} of {case.cfg.num_seqs} sequences of the same workload, one full step "
-                      f"(copies, new-token write, fp64 decode), best of {reps}"}
+                      f"(copies, new-token write, fp64 decode), best of {reps}",
+            "single_thread": {"value": round(sample1.kv_bytes() / dt1 / 1e9, 4), "unit": "GB/s",
+                              "seqs_per_s": round(n1 / dt1, 3),
+                              "sample": f"first {n1} sequences, one step, one run"}}
 
 
 def run_reference(args, world, rank):
@@ -808,7 +834,7 @@ def run_reference(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": cfg.name, "description": cfg.description, "sample_seqs_per_step": n},
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": o.num_threads, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": o.num_threads, "kind": "oracle", "cpu": cpu_model(),
                          "sample": desc},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

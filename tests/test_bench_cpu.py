@@ -61,3 +61,14 @@ def test_reference_arm_decode():
     d = _reference_line("tiny")
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["metric"] == bench.METRIC
     assert d["value"] > 0 and d["config"]["workload"] == "tiny"
+
+
+def test_cpu_baseline_reports_all_threads_and_one():
+    case = inputs.make_case("tiny")
+    d = bench.cpu_baseline(case, budget_s=2.0)
+    assert d["kind"] == "oracle" and d["unit"] == "GB/s" and d["value"] > 0 and d["cores"] >= 1
+    assert isinstance(d["cpu"], str) and d["cpu"]
+    one = d["single_thread"]
+    assert one["unit"] == "GB/s" and one["value"] > 0 and one["seqs_per_s"] > 0
+    import oracle
+    assert oracle.get().num_threads == d["cores"]   # thread count restored
