@@ -74,3 +74,20 @@ def test_case_structure(name, lens):
         (b, lb), = owners[dst]
         assert int(case.shared_block_tables[b, lb]) == src
         assert sum(int(r[lb]) == src for r in case.shared_block_tables.tolist()) > 1
+
+
+def test_prefill_recipe_and_flop_count():
+    """16 chunks of 512 tokens after prefixes drawn U[0, 1536] (seed 1007); the
+    metric's unit, 4*Hq*D per causally visible (query, key) pair, from its
+    closed form: a chunk of n queries after L-n cached tokens sees
+    n(L-n) + n(n+1)/2 pairs."""
+    case = inputs.make_prefill_case("llama3_8b_prefill")
+    cfg = case.cfg
+    assert cfg.seed == 1007 and cfg.num_seqs == 16
+    qsl = case.query_start_loc.tolist()
+    assert qsl == [512 * i for i in range(17)] and case.max_query_len == 512 and case.num_tokens == 8192
+    L = case.context_lens.tolist()
+    assert all(512 <= x <= 512 + 1536 for x in L) and (min(L), max(L)) == (595, 1888)
+    pairs = sum(512 * (x - 512) + 512 * 513 // 2 for x in L)
+    assert case.flops() == 4 * cfg.num_heads * cfg.head_dim * pairs == 130291859456
+    assert case.kv_bytes_attended() == sum(L) * cfg.num_kv_heads * cfg.head_dim * 2 * 2
