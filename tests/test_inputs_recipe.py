@@ -91,3 +91,19 @@ def test_prefill_recipe_and_flop_count():
     pairs = sum(512 * (x - 512) + 512 * 513 // 2 for x in L)
     assert case.flops() == 4 * cfg.num_heads * cfg.head_dim * pairs == 130291859456
     assert case.kv_bytes_attended() == sum(L) * cfg.num_kv_heads * cfg.head_dim * 2 * 2
+
+
+KV_BYTES = {"tiny": 409600, "llama2_7b": 1054343168, "llama3_8b_gqa": 1206407168, "shared_prefix": 679071744,
+            "long_context": 1073741824, "llama3_8b_gqa_fp8": 608784384}
+
+
+@pytest.mark.parametrize("name", sorted(KV_BYTES))
+def test_decode_metric_bytes(name):
+    """The decode metric's algorithmic bytes: every attended token's K and V
+    rows once, sum_b L_b * Hkv * 2 * D * element size (1 byte for E4M3)."""
+    cfg = inputs.CONFIGS[name]
+    es = 1 if cfg.kv_dtype == "fp8_e4m3" else {"f32": 4, "f16": 2, "bf16": 2}[cfg.dtype]
+    assert TOTALS[name] * cfg.num_kv_heads * 2 * cfg.head_dim * es == KV_BYTES[name]
+    lens = {"tiny": None, "shared_prefix": [1040, 1100, 1300]}.get(name, [1, 16, 17, 300])
+    small = inputs.make_case(name, lens=lens, with_post=False)
+    assert small.kv_bytes() == int(small.context_lens.sum()) * cfg.num_kv_heads * 2 * cfg.head_dim * es
