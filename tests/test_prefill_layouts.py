@@ -1,0 +1,131 @@
+"""The paged-prefill kernel's operand layouts, emulated on the CPU.
+
+csrc/pa_prefill.cuh stages Q with generic 16-byte stores that apply the
+128-byte swizzle themselves, lands K and V tiles with TMA boxes (one 128-byte
+half of 16 token rows per cache block, hardware swizzle), and hands the tensor
+cores shared-memory descriptors (start address, leading / stride byte offsets)
+for S = Q K^T (both operands K-major) and O += P V (V MN-major).  The 128-byte
+swizzle exchanges the 16-byte chunks of each 128-byte row by the row's index
+within its 1024-byte atom.  Tile elements here are unique 16-bit identifiers,
+so every operand the descriptors describe must read back exactly the matrix
+the product needs.  Also checked: where P's two 16-bit parts land in tensor
+memory for the products that read them, and the accuracy of the hi + lo split.
+"""
+import numpy as np
+
+ROWS, KV, HALF_ROWS = 128, 64, 128 * 128       # query rows, KV tile tokens, bytes of one Q half
+KV_HALF = KV * 128                              # bytes of one 64-element half of a KV tile
+
+
+def swz(a):
+    """Physical address of logical address a under the 128-byte swizzle (1024-byte atoms)."""
+    return a ^ (((a >> 7) & 7) << 4)
+
+
+def read16(sm, addr):
+    addr = np.asarray(addr)
+    return sm[addr].astype(np.uint32) | (sm[addr + 1].astype(np.uint32) << 8)
+
+
+def read_kmajor(sm, start, sbo, rows):
+    """A K-major operand of `rows` x 16 elements: 8-row groups sbo bytes apart, 128-byte rows."""
+    r = np.arange(rows)[:, None]
+    k = np.arange(16)[None, :]
+    return read16(sm, swz(start + (r % 8) * 128 + (r // 8) * sbo + 2 * k))
+
+
+def read_mnmajor(sm, start, lbo, sbo, nmn):
+    """An MN-major operand of 16 (K) x nmn elements: 64-element MN groups lbo bytes apart,
+    consecutive K in consecutive 128-byte rows, 8-row K groups sbo bytes apart."""
+    k = np.arange(16)[:, None]
+    mn = np.arange(nmn)[None, :]
+    return read16(sm, swz(start + (mn % 64) * 2 + (mn // 64) * lbo + (k % 8) * 128 + (k // 8) * sbo))
+
+
+def ids(rows, cols, base):
+    return (base + np.arange(rows * cols, dtype=np.uint32).reshape(rows, cols)) & 0xFFFF
+
+
+def put16(sm, addr, v):
+    sm[addr], sm[addr + 1] = v & 0xFF, v >> 8
+
+
+def test_q_staging_and_qk_descriptors():
+    Q = ids(ROWS, 128, 1)
+    sm = np.zeros(2 * HALF_ROWS, np.uint8)
+    for row in range(ROWS):                         # the kernel's Q store: chunk c of a row, swizzled by hand
+        for c in range(16):
+            base = (c >> 3) * HALF_ROWS + row * 128 + (((c & 7) ^ (row & 7)) << 4)
+            for e in range(8):
+                put16(sm, base + 2 * e, Q[row, 8 * c + e])
+    for kk in range(8):                             # a_qk + ((kk >> 2) * half + (kk & 3) * 32)
+        start = (kk >> 2) * HALF_ROWS + (kk & 3) * 32
+        assert np.array_equal(read_kmajor(sm, start, 1024, ROWS), Q[:, 16 * kk:16 * kk + 16])
+
+
+def _tma_tile(X_blocks):
+    """A KV tile from 4 cache blocks (16 tokens x 128 elements each) placed as the TMA
+    boxes do: half h of block bi at h * KV_HALF + bi * 16 * 128, rows of 128 bytes, swizzled."""
+    sm = np.zeros(2 * KV_HALF, np.uint8)
+    for bi, X in enumerate(X_blocks):
+        for h in range(2):
+            dst = h * KV_HALF + bi * 16 * 128
+            for t in range(16):
+                for e in range(64):
+                    put16(sm, swz(dst + t * 128 + 2 * e), X[t, 64 * h + e])
+    return sm
+
+
+def test_kv_tiles_and_product_descriptors():
+    blocks_k = [ids(16, 128, 1000 * (i + 1)) for i in range(4)]
+    blocks_v = [ids(16, 128, 7000 + 1000 * i) for i in range(4)]
+    K, V = np.vstack(blocks_k), np.vstack(blocks_v)            # logical 64 x 128 tiles
+    smk, smv = _tma_tile(blocks_k), _tma_tile(blocks_v)
+    for kk in range(8):                                        # QK: B = K tile, K-major, N = 64
+        start = (kk >> 2) * KV_HALF + (kk & 3) * 32
+        assert np.array_equal(read_kmajor(smk, start, 1024, KV), K[:, 16 * kk:16 * kk + 16])
+    for kk in range(KV // 16):                                 # PV: B = V tile, MN-major, N = 128 (head_dim)
+        got = read_mnmajor(smv, kk * 16 * 128, KV_HALF, 1024, 128)
+        assert np.array_equal(got, V[16 * kk:16 * kk + 16, :])
+
+
+def test_p_columns_in_tensor_memory():
+    """The softmax stores P(j) over S(j): hi pairs (tokens 2k, 2k+1) at column k,
+    lo pairs at column 32 + k, the lower token in the low half.  The product for
+    tokens 16kk..16kk+15 of part p reads columns p*32 + 8kk .. + 7."""
+    col_of = {}
+    for part in range(2):
+        for k in range(32):
+            for h in range(2):
+                col_of[(part, 2 * k + h)] = (part * 32 + k, h)
+    for part in range(2):
+        for kk in range(KV // 16):
+            cols = [part * 32 + kk * 8 + c for c in range(8)]
+            tokens = [(c - part * 32) * 2 + h for c in cols for h in range(2)]
+            assert tokens == list(range(16 * kk, 16 * kk + 16))
+            assert all(col_of[(part, t)][0] in cols for t in tokens)
+
+
+def test_hi_lo_split_accuracy():
+    """hi = p truncated to bf16, lo = the exact remainder truncated to bf16:
+    |p - hi - lo| < 2^-15 |p| over p in (0, 2^8] (the lazy-rescale range)."""
+    rng = np.random.default_rng(5)
+    p = np.concatenate([rng.uniform(0, 1, 200000), rng.uniform(1, 256, 50000),
+                        2.0 ** rng.uniform(-40, 0, 50000)]).astype(np.float32)
+    p = p[p > 0]
+    trunc = lambda x: (x.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    hi = trunc(p)
+    rem = (p - hi).astype(np.float32)              # exact: hi holds p's top bits
+    assert np.array_equal(rem.astype(np.float64), p.astype(np.float64) - hi.astype(np.float64))
+    lo = trunc(rem)
+    err = np.abs(p.astype(np.float64) - hi.astype(np.float64) - lo.astype(np.float64))
+    assert (err < 2.0 ** -15 * p.astype(np.float64)).all()
+    # one 16-bit part alone would not do: its error reaches 2^-8 relative
+    assert (np.abs(p.astype(np.float64) - hi.astype(np.float64)) / p).max() > 2.0 ** -9
+
+
+def test_emulation_catches_a_wrong_stride():
+    """The V operand read with the K-major stride (lbo = 16) is wrong."""
+    blocks_v = [ids(16, 128, 7000 + 1000 * i) for i in range(4)]
+    V, smv = np.vstack(blocks_v), _tma_tile(blocks_v)
+    assert not np.array_equal(read_mnmajor(smv, 0, 16, 1024, 128), V[0:16, :])
