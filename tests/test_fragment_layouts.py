@@ -194,3 +194,15 @@ def test_emulation_catches_a_wrong_swizzle():
     mi, ri = LANES >> 3, LANES & 7
     addrs = [plain(ri[l] + 8 * (mi[l] & 1), 2 * 0 + (mi[l] >> 1)) for l in range(32)]
     assert not conflict_free(addrs)
+
+
+def test_tile_offset_is_where_the_tma_box_lands():
+    """The decode tiles arrive by TMA (box {128 B, 1, 1, 16 tokens, 1} per
+    128-byte half, 128-byte swizzle: 16-byte chunk j of a 128-byte row moves to
+    j ^ (row within the 1024-byte atom)); tile_offset must name the same bytes."""
+    def swizzled(logical):
+        return logical ^ (((logical >> 7) & 7) << 4)
+    for t in range(T):
+        for c in range(16):
+            half, j = c >> 3, c & 7
+            assert tile_offset(t, c) == swizzled(half * T * 128 + t * 128 + j * 16)
