@@ -199,6 +199,69 @@ def barrier(world: int):
         dist.barrier()
 
 
+# ------------------------------------------------------------------ timing helpers
+def percentile(xs, q: float) -> float:
+    """The q-th percentile of xs (linear interpolation between order statistics)."""
+    ys = sorted(xs)
+    if not ys:
+        return float("nan")
+    k = (len(ys) - 1) * q / 100.0
+    lo = int(math.floor(k))
+    hi = min(lo + 1, len(ys) - 1)
+    return ys[lo] + (ys[hi] - ys[lo]) * (k - lo)
+
+
+def spread_line(ms, work, peak, unit, scale, what):
+    """Mean / median / p10 / p90 of per-call times and the work rate at the median."""
+    med = statistics.median(ms)
+    rate = work / (med * 1e-3) / scale
+    return {"calls": len(ms), "ms_mean": round(statistics.mean(ms), 5), "ms_median": round(med, 5),
+            "ms_p10": round(percentile(ms, 10), 5), "ms_p90": round(percentile(ms, 90), 5),
+            "achieved_at_median": round(rate, 2), "unit": unit, "frac_at_median": round(rate / peak, 4),
+            "what": what}
+
+
+def l2_flushed_calls(pre, call, n, stream, device):
+    """Per-call times of ``call`` (events on its stream), each call preceded by
+    ``pre`` and by a 256 MiB write (2x the L2) outside the events."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        pre()
+        flush.fill_(i & 0xff)
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    del flush
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def stream_read_probe(device, nbytes: int = 2 << 30, reps: int = 20):
+    """Read-only bandwidth of the library's plain streaming-read kernel
+    (pa_stream_read) over a buffer 16x the L2, median of ``reps`` timed reads."""
+    from paged_kv_cache_464_b200 import capi
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    buf.fill_(1)
+    sink = torch.zeros(1, dtype=torch.int64, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        capi.stream_read(buf, sink)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record(stream)
+        capi.stream_read(buf, sink)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    del buf
+    med = statistics.median(ms)
+    return {"kernel": "pa_stream_read (16-byte streaming loads, 8 CTAs x 256 threads per SM)",
+            "bytes": nbytes, "ms_median": round(med, 5), "gbs_median": round(nbytes / (med * 1e-3) / 1e9, 1),
+            "gbs_best": round(nbytes / (min(ms) * 1e-3) / 1e9, 1), "reps": reps}
+
+
 # ------------------------------------------------------------------ our arm
 class Step:
     """The device buffers of one workload and the step's calls through the C ABI."""
@@ -264,6 +327,36 @@ class Step:
         self.pre()
         self.decode()
 
+    def raw_calls(self, t, out, stream):
+        """The step as (C function, argument tuple) pairs over the tensors ``t``
+        (name -> device tensor: q, key, value, slots, pairs, bt, cl) and ``out``,
+        arguments marshalled once, for a loop that calls the C ABI directly."""
+        r, c, case = self.pa.raw, self.case.cfg, self.case
+        nb, bs, hkv, d = self.k.shape
+        s = stream.cuda_stream
+        ws, wsb = self.ws.data_ptr(), self.ws.numel()
+        S, hq, mbs = c.num_seqs, c.num_heads, t["bt"].shape[1]
+        calls = []
+        if self.has_pairs:
+            calls.append((r.pa_copy_blocks, (self.k.data_ptr(), self.v.data_ptr(), t["pairs"].data_ptr(),
+                                             t["pairs"].shape[0], nb, bs, hkv, d, self.pa.DTYPE_CODE[self.q.dtype]
+                                             if not self.fp8 else self.pa.FP8, s)))
+        if self.fp8:
+            qd = self.pa.DTYPE_CODE[self.q.dtype]
+            calls.append((r.pa_reshape_and_cache_fp8, (t["key"].data_ptr(), t["value"].data_ptr(), self.k.data_ptr(),
+                                                       self.v.data_ptr(), t["slots"].data_ptr(), t["key"].shape[0], nb,
+                                                       bs, hkv, d, qd, self.kv_scale, self.kv_scale, s)))
+            calls.append((r.pa_decode_fp8, (out.data_ptr(), t["q"].data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                                            self.kv_scale, self.kv_scale, t["bt"].data_ptr(), mbs, t["cl"].data_ptr(),
+                                            S, hq, self.maxL, case.scale, self.P, ws, wsb, nb, bs, hkv, d, qd, s)))
+        else:
+            dt = self.pa.DTYPE_CODE[self.q.dtype]
+            calls.append((r.pa_decode_append, (out.data_ptr(), t["q"].data_ptr(), t["key"].data_ptr(),
+                                               t["value"].data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                                               t["bt"].data_ptr(), mbs, t["cl"].data_ptr(), S, hq, self.maxL,
+                                               case.scale, self.P, ws, wsb, nb, bs, hkv, d, dt, s)))
+        return calls
+
     # the same step as three separate calls (pa_copy_blocks, pa_reshape_and_cache, pa_decode)
     def separate(self):
         if self.fp8:
@@ -318,6 +411,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
 
+    # ---- the same calls with L2 flushed before each (a 256 MiB write between
+    # steps, outside the events): shows the figures do not come from L2 reuse
+    flushed_ms = l2_flushed_calls(step.pre, step.decode, min(args.steps, 200), stream, device)
+
     # the same K steps as three separate calls, for comparison
     for _ in range(args.warmup):
         step.separate()
@@ -340,6 +437,9 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
     wall_soak = time.time()
     sampler.stop()
+
+    # ---- read-only bandwidth of a plain streaming-read kernel (context for the fraction)
+    read_probe = stream_read_probe(device)
 
     # ---- end to end through the public API from pinned host buffers
     e2e = run_e2e(case, step, args.steps, args.warmup, device)
@@ -410,10 +510,18 @@ def run_ours(args, world, rank, local):
             "traffic": traffic,
             "decode_ms_mean": round(dec_avg, 5),
             "decode_ms_median": round(statistics.median(dec_ms), 5),
+            "decode_ms_p10": round(percentile(dec_ms, 10), 5),
+            "decode_ms_p90": round(percentile(dec_ms, 90), 5),
+            "l2_flushed": spread_line(flushed_ms, kv_bytes, peak, "GB/s", 1e9,
+                                      "the same calls, each after a 256 MiB write that evicts L2"),
+            "read_probe": read_probe,
         },
         "e2e": {"value": round(total_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                "ms_per_step": round(e2e_ms / args.steps, 5)},
+                "ms_per_step": round(e2e_ms / args.steps, 5),
+                "host_us_per_step": e2e["host_us"],
+                "frac_of_value": round(max_ms / e2e_ms, 4),
+                "path": e2e["path"]},
         "gpu_launches": step.launches(fused=True) * args.steps,
         "clocks": clocks,
     }
@@ -454,6 +562,20 @@ class PrefillStep:
     def __call__(self):
         self.write()
         self.attend()
+
+    def raw_calls(self, t, out, stream):
+        """The step as (C function, argument tuple) pairs over the tensors ``t``
+        (q, key, value, slots, bt, cl, qsl) and ``out``; see Step.raw_calls."""
+        r, c = self.pa.raw, self.case.cfg
+        nb, bs, hkv, d = self.kc.shape
+        dt = self.pa.DTYPE_CODE[self.q.dtype]
+        s = stream.cuda_stream
+        return [(r.pa_reshape_and_cache, (t["key"].data_ptr(), t["value"].data_ptr(), self.kc.data_ptr(),
+                                          self.vc.data_ptr(), t["slots"].data_ptr(), t["key"].shape[0], nb, bs, hkv,
+                                          d, dt, s)),
+                (r.pa_prefill, (out.data_ptr(), t["q"].data_ptr(), self.kc.data_ptr(), self.vc.data_ptr(),
+                                t["bt"].data_ptr(), t["bt"].shape[1], t["cl"].data_ptr(), t["qsl"].data_ptr(),
+                                c.num_seqs, c.num_heads, self.max_query_len, self.case.scale, nb, bs, hkv, d, dt, s))]
 
 
 def chunk_slots(case: inputs.PrefillCase) -> torch.Tensor:
@@ -502,6 +624,7 @@ def run_prefill(args, world, rank, local):
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     att_ms = [a.elapsed_time(b) for a, b in ev]
+    flushed_ms = l2_flushed_calls(step.write, step.attend, min(args.steps, 200), stream, device)
 
     soak_until = wall0 + 2.5
     while time.time() < soak_until:
@@ -565,10 +688,17 @@ def run_prefill(args, world, rank, local):
             "traffic": profiled_traffic(args.workload, kernel="pa_prefill"),
             "prefill_ms_mean": round(att_avg, 5),
             "prefill_ms_median": round(statistics.median(att_ms), 5),
+            "prefill_ms_p10": round(percentile(att_ms, 10), 5),
+            "prefill_ms_p90": round(percentile(att_ms, 90), 5),
+            "l2_flushed": spread_line(flushed_ms, flops, peak, "TFLOP/s", 1e12,
+                                      "the same calls, each after a 256 MiB write that evicts L2"),
         },
         "e2e": {"value": round(total_flops * args.steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                "ms_per_step": round(e2e_ms / args.steps, 5)},
+                "ms_per_step": round(e2e_ms / args.steps, 5),
+                "host_us_per_step": e2e["host_us"],
+                "frac_of_value": round(max_ms / e2e_ms, 4),
+                "path": e2e["path"]},
         "gpu_launches": 2 * args.steps,
         "clocks": sampler.summary(wall0, wall_soak),
     }
@@ -579,11 +709,11 @@ def run_prefill(args, world, rank, local):
 
 def run_e2e_prefill(step: PrefillStep, steps, warmup):
     """Per step: q, the chunk K/V rows, slots and tables host->device from pinned
-    memory, the step through the public API, out device->host."""
+    memory, the step through the C ABI, out device->host."""
     case = step.case
     host = {"q": case.q, "key": step.key_host, "value": step.value_host, "slots": step.slots_host,
             "bt": case.block_tables, "cl": case.context_lens, "qsl": case.query_start_loc}
-    return pipelined_e2e(step, {k: t.pin_memory() for k, t in host.items()}, steps, warmup)
+    return pipelined_e2e(step, host, step.out, steps, warmup)
 
 
 def _oracle_prefill(o, case):
@@ -646,20 +776,49 @@ def run_reference_prefill(args, world, rank):
     }
 
 
-def pipelined_e2e(step, host, steps, warmup):
-    """End to end through the public API: every step copies its inputs `host`
-    (step attribute name -> pinned host tensor) to the device, runs `step()`
-    and copies `step.out` back into pinned host memory.  Two sets of device
-    inputs and outputs alternate between steps, with one copy stream per
-    direction, so that step k's copies overlap the kernels of step k-1 (as a
-    serving loop would run them); every copy of every timed step lies inside
-    the timed region."""
-    names = list(host)
+class PackedInputs:
+    """All of a step's input tensors in ONE pinned host buffer, and two device
+    buffers of the same layout (each tensor at a 256-byte-aligned offset), so a
+    step's inputs move with one host->device copy; views into a device buffer
+    feed the calls."""
+
+    def __init__(self, tensors, device):
+        self.offsets, off = {}, 0
+        for n, t in tensors.items():
+            self.offsets[n] = off
+            off += (t.numel() * t.element_size() + 255) // 256 * 256
+        self.nbytes = off
+        self.host = torch.zeros(off, dtype=torch.uint8).pin_memory()
+        for n, t in tensors.items():
+            o, nb = self.offsets[n], t.numel() * t.element_size()
+            self.host[o:o + nb].copy_(t.contiguous().reshape(-1).view(torch.uint8))
+        self.dev = [torch.empty(off, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.views = []
+        for buf in self.dev:
+            v = {}
+            for n, t in tensors.items():
+                o, nb = self.offsets[n], t.numel() * t.element_size()
+                v[n] = buf[o:o + nb].view(t.dtype).view(t.shape)
+            self.views.append(v)
+
+
+def pipelined_e2e(step, host, out_like, steps, warmup):
+    """End to end through the C ABI: every step copies its inputs ``host``
+    (name -> host tensor, packed into one pinned buffer) to the device in one
+    copy, makes the step's C calls (arguments marshalled once, the call made
+    directly, no per-call Python checks) and copies the output back into pinned
+    host memory.  Two sets of device inputs and outputs alternate between steps,
+    with one copy stream per direction, so that step k's copies overlap the
+    kernels of step k-1 (as a serving loop would run them); every copy of every
+    timed step lies inside the timed region.  Also reports the host time of
+    issuing a step (a short burst timed with the GPU idle at its start)."""
     compute = torch.cuda.current_stream()
+    device = out_like.device
     h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
-    bufs = [{n: getattr(step, n) for n in names}, {n: torch.empty_like(getattr(step, n)) for n in names}]
-    outs = [step.out, torch.empty_like(step.out)]
-    out_host = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
+    packed = PackedInputs(host, device)
+    outs = [torch.empty_like(out_like) for _ in range(2)]
+    out_host = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory() for _ in range(2)]
+    calls = [step.raw_calls(packed.views[i], outs[i], compute) for i in range(2)]
     loaded = [torch.cuda.Event() for _ in range(2)]     # inputs of set i on the device
     consumed = [torch.cuda.Event() for _ in range(2)]   # kernels that read set i (and write its output) done
     drained = [torch.cuda.Event() for _ in range(2)]    # output of set i copied to the host
@@ -668,15 +827,14 @@ def pipelined_e2e(step, host, steps, warmup):
         i = k & 1
         h2d_s.wait_event(consumed[i])                   # the step two back is done with these inputs
         with torch.cuda.stream(h2d_s):
-            for n in names:
-                bufs[i][n].copy_(host[n], non_blocking=True)
+            packed.dev[i].copy_(packed.host, non_blocking=True)
         loaded[i].record(h2d_s)
         compute.wait_event(loaded[i])
         compute.wait_event(drained[i])                  # its output buffer has been read out
-        for n in names:
-            setattr(step, n, bufs[i][n])
-        step.out = outs[i]
-        step()
+        for fn, a in calls[i]:
+            rc = fn(*a)
+            if rc != 0:
+                raise RuntimeError(f"{fn.__name__}: status {rc}")
         consumed[i].record(compute)
         d2h_s.wait_event(consumed[i])
         with torch.cuda.stream(d2h_s):
@@ -696,27 +854,31 @@ def pipelined_e2e(step, host, steps, warmup):
 
     loop(max(2, warmup))
     torch.cuda.synchronize()
+    burst = min(steps, 32)
+    t0 = time.perf_counter()
+    loop(burst)
+    host_us = (time.perf_counter() - t0) * 1e6 / burst
+    torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(compute)
     loop(steps)
     b.record(compute)
     torch.cuda.synchronize()
-    for n in names:
-        setattr(step, n, bufs[0][n])
-    step.out = outs[0]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host[0].numel() * out_host[0].element_size()
-    return {"ms": a.elapsed_time(b), "h2d": h2d, "d2h": d2h, "last_out_host": out_host[(steps - 1) & 1]}
+    return {"ms": a.elapsed_time(b), "h2d": packed.nbytes, "d2h": d2h, "host_us": round(host_us, 2),
+            "last_out_host": out_host[(steps - 1) & 1],
+            "path": "one packed pinned->device copy, direct C-ABI calls, one device->pinned copy per step; "
+                    "two buffer sets alternate so copies overlap the previous step's kernels"}
 
 
 def run_e2e(case, step, steps, warmup, device):
     """Per step: inputs host->device from pinned memory, the step through the
-    public API, the output device->host into pinned memory."""
+    C ABI, the output device->host into pinned memory."""
     host = {"q": case.q, "key": case.key, "value": case.value, "slots": case.slot_mapping,
             "bt": case.block_tables, "cl": case.context_lens}
     if step.has_pairs:
         host["pairs"] = case.block_mapping
-    return pipelined_e2e(step, {k: t.pin_memory() for k, t in host.items()}, steps, warmup)
+    return pipelined_e2e(step, host, step.out, steps, warmup)
 
 
 # ------------------------------------------------------------------ oracle timings

@@ -21,8 +21,13 @@
  * --------------------------------
  * - Every pointer argument except `stream` and the `detail` out-parameter of
  *   pa_get_device_error is DEVICE memory owned by the caller.  The library
- *   allocates no device or host memory and keeps no state across calls except
- *   one device error word per GPU (see pa_get_device_error).
+ *   allocates no device or host memory at run time.  What it keeps across
+ *   calls: one device error word per GPU (see pa_get_device_error); the SM
+ *   count of each GPU (queried once, to size grids); and two arrays that exist
+ *   from load time in every GPU that loads the library -- the 64 MiB split-K
+ *   scratch of pa_decode_static_workspace, which keeps the last such call's
+ *   contents, and the error word.  pa_test_stall_next_launch arms a one-shot
+ *   host-side flag (tests only).
  * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *   NULL = the legacy default stream).  The returned status covers host-side
  *   argument checks and the launch itself (cudaGetLastError).  Problems that
@@ -71,7 +76,8 @@ typedef enum {
   PA_DEV_BAD_SLOT = 2,         /* slot >= num_blocks * block_size; detail = the slot */
   PA_DEV_COPY_CONFLICT = 3,    /* copy pair skipped (dst repeated or read by a pair); detail = pair index */
   PA_DEV_BAD_CONTEXT_LEN = 4,  /* context_len < 0, > max_context_len or > table capacity; detail = seq */
-  PA_DEV_WAIT_TIMEOUT = 5,     /* an internal bounded wait gave up; detail = CTA index */
+  PA_DEV_WAIT_TIMEOUT = 5,     /* an internal bounded wait gave up; detail = linear CTA index
+                                  (blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) */
 } pa_device_error_t;
 
 /*
@@ -255,11 +261,19 @@ pa_status_t pa_prefill(void *out, const void *q, const void *k_cache, const void
  * block dst.  A pair is skipped and recorded as PA_DEV_BAD_BLOCK_ID if an id
  * is outside [0, num_blocks), or as PA_DEV_COPY_CONFLICT if its dst is the dst
  * of another pair or the src of any pair (itself included); all other pairs
- * are carried out, independently of their order.  The conflict check reads
- * all pairs from every CTA: cost O(num_pairs^2) reads of 16 bytes.
- * Errors: PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_CUDA.
- * num_pairs == 0 is a no-op.
+ * are carried out, independently of their order.
+ * Cost of the conflict check: each of the kernel's CTAs (up to 2 per SM, more
+ * for large batches: one per 256 pairs) reads the mapping once through shared
+ * memory, and the pairs are compared num_pairs^2 times in shared memory in
+ * all.  num_pairs is capped at PA_MAX_COPY_PAIRS so that this stays bounded
+ * (at the cap, about the time of copying the blocks themselves for 8 KV heads
+ * of 256-byte rows); copy-on-write batches are far smaller in practice (one
+ * block per sequence that writes into a shared block).
+ * Errors: PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE (incl. num_pairs < 0 or >
+ * PA_MAX_COPY_PAIRS), PA_ERR_ALIGN, PA_ERR_CUDA.  num_pairs == 0 is a no-op.
  */
+#define PA_MAX_COPY_PAIRS 65536
+
 pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
                            int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
                            pa_dtype_t dtype, void *stream);
@@ -288,9 +302,18 @@ pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_ma
  * fits; 4096 sequences of that shape would not).  The call allocates no device
  * or host memory: no cudaMalloc, no cudaFree, no allocating library routine.
  *
- * Set-up: the first accepted call on a device (that device current) looks up
- * the array's device address with cudaGetSymbolAddress and caches it; make
- * that first call before any stream capture.  Later calls do no set-up.
+ * Checks: every check of pa_decode, in pa_decode's order, comes first (so a
+ * call that is invalid in another way returns what pa_decode returns); then a
+ * call whose split-K scratch need exceeds PA_STATIC_WORKSPACE_BYTES returns
+ * PA_ERR_WORKSPACE without launching anything.
+ *
+ * Set-up: every call that needs scratch (one that splits a sequence) looks up
+ * the array's address on the current device with cudaGetSymbolAddress, which
+ * allocates nothing; the address is never cached, so a cudaDeviceReset (which
+ * gives the device a new context and a new copy of the array) needs nothing
+ * from the caller.  The first lookup on a device may load the library's
+ * device code there, so make the first call on each device before any stream
+ * capture.
  *
  * Sharing: every call on a device uses the same array, which keeps the last
  * call's contents.  Nothing in it needs clearing between calls (each call
@@ -304,6 +327,35 @@ pa_status_t pa_decode_static_workspace(void *out, const void *q, const void *k_c
                                        int max_context_len, float scale, int partition_size,
                                        int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
                                        pa_dtype_t dtype, void *stream);
+
+/*
+ * pa_stream_read -- measurement helper with no counterpart on the source
+ * pages: read `bytes` of device memory once, as a plain streaming read (16-byte
+ * loads, eight 256-thread CTAs per SM), and XOR every 8-byte little-endian word
+ * of it into *sink (device memory, 8-byte aligned; the caller zeroes it first
+ * if it wants the XOR itself).  Its duration gives the read-only bandwidth the
+ * decode kernels are measured against.  bytes must be a multiple of 16 and buf
+ * 16-byte aligned.  Errors: PA_ERR_SHAPE, PA_ERR_NULL, PA_ERR_ALIGN,
+ * PA_ERR_CUDA.  bytes == 0 is a no-op.
+ */
+pa_status_t pa_stream_read(const void *buf, size_t bytes, uint64_t *sink, void *stream);
+
+/*
+ * pa_test_stall_next_launch -- test hook for the bounded-wait error path (no
+ * counterpart on the source pages; ordinary callers never need it).
+ *
+ * Arms a one-shot flag in the host library: the next launch of `kernel`
+ * (0 = the decode partition kernel of any pa_decode* call, 1 = pa_prefill),
+ * from any thread, carries it and clears it.  In that launch, CTA `cta` (the
+ * linear index of PA_DEV_WAIT_TIMEOUT) leaves one of its tile copies unissued
+ * -- no copy and no barrier arrival, so nothing is in flight for it -- and its
+ * waits give up after 1 ms instead of 2 s.  Its wait on the missing tile runs
+ * out, it records PA_DEV_WAIT_TIMEOUT with detail = `cta`, lets its other
+ * copies in flight land, and returns without writing its output rows; every
+ * other CTA runs normally.  The GPU context stays usable.  cta = -1 disarms.
+ * Errors: PA_ERR_SHAPE for an unknown kernel or cta < -1.
+ */
+pa_status_t pa_test_stall_next_launch(int kernel, int64_t cta);
 
 /*
  * pa_get_device_error -- synchronise `stream`, then return the first problem a

@@ -43,6 +43,10 @@ _lib.pa_prefill.restype = _I
 _lib.pa_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _F, _I64, _I, _I, _I, _I, _P]
 _lib.pa_copy_blocks.restype = _I
 _lib.pa_copy_blocks.argtypes = [_P, _P, _P, _I, _I64, _I, _I, _I, _I, _P]
+_lib.pa_stream_read.restype = _I
+_lib.pa_stream_read.argtypes = [_P, _SZ, _P, _P]
+_lib.pa_test_stall_next_launch.restype = _I
+_lib.pa_test_stall_next_launch.argtypes = [_I, _I64]
 _lib.pa_get_device_error.restype = _I
 _lib.pa_get_device_error.argtypes = [_P, ctypes.POINTER(_I64), _I]
 _lib.pa_status_string.restype = ctypes.c_char_p
@@ -50,7 +54,8 @@ _lib.pa_status_string.argtypes = [_I]
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode",
             "pa_decode_append", "pa_decode_static_workspace", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_prefill",
-            "pa_copy_blocks", "pa_get_device_error", "pa_status_string"]
+            "pa_copy_blocks", "pa_stream_read", "pa_test_stall_next_launch", "pa_get_device_error", "pa_status_string"]
+MAX_COPY_PAIRS = 65536       # PA_MAX_COPY_PAIRS in include/pa.h
 STATIC_WORKSPACE_BYTES = 64 << 20   # PA_STATIC_WORKSPACE_BYTES in include/pa.h
 
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
@@ -320,6 +325,24 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: tor
     _check(_lib.pa_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
                                _dev(block_mapping, "block_mapping") if P else None, P, nb, bs, hkv, d, dt,
                                _stream(stream)), "pa_copy_blocks")
+
+
+def stream_read(buf: torch.Tensor, sink: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Read every byte of ``buf`` once (a plain streaming read, for measuring the
+    read-only bandwidth); XORs its 8-byte words into ``sink`` (one int64 on the device)."""
+    if sink.dtype != torch.int64 or sink.numel() != 1:
+        raise ValueError("sink must be one int64")
+    _check(_lib.pa_stream_read(_dev(buf, "buf"), buf.numel() * buf.element_size(), _dev(sink, "sink"),
+                               _stream(stream)), "pa_stream_read")
+
+
+def test_stall_next_launch(kernel: str, cta: int) -> None:
+    """Test hook: the next launch of ``kernel`` ("decode" or "prefill") leaves
+    one copy of CTA ``cta`` unissued, so that CTA's bounded wait runs out
+    (PA_DEV_WAIT_TIMEOUT, detail = cta) within about a millisecond; ``cta=-1``
+    disarms."""
+    _check(_lib.pa_test_stall_next_launch({"decode": 0, "prefill": 1}[kernel], int(cta)),
+           "pa_test_stall_next_launch")
 
 
 def get_device_error(clear: bool = True, stream: Optional[torch.cuda.Stream] = None):

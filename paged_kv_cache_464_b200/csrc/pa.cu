@@ -5,6 +5,7 @@
 // device linking.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -16,9 +17,16 @@
 #include "pa_cache_ops.cuh"
 #include "pa_decode.cuh"
 #include "pa_prefill.cuh"
+#include "pa_probe.cuh"
 
 #ifndef PA_PROGRAMMATIC_LAUNCH
 #define PA_PROGRAMMATIC_LAUNCH 1
+#endif
+// Split sequences: 1 = the last partition CTA of each (sequence, KV head)
+// combines the partials (one launch, plus a tiny counter-zeroing kernel);
+// 0 = a separate reduce kernel after the partition kernel.
+#ifndef PA_FUSED_COMBINE
+#define PA_FUSED_COMBINE 1
 #endif
 
 namespace {
@@ -27,6 +35,27 @@ using pa::kBlockSize;
 using pa::kRowBytes;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Streaming multiprocessors of the current device, queried once per device
+// (grids of the cache operations and the reduce are sized from it).  Falls
+// back to 148 (a full B200) if the query fails.
+constexpr int kMaxDevices = 128;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Test hook (pa_test_stall_next_launch): armed by a test, consumed by the next
+// decode or prefill launch of the armed kind; 0 = not armed.
+std::atomic<int> g_stall_decode{0};
+std::atomic<int> g_stall_prefill{0};
 
 int elem_bytes(pa_dtype_t dt) {
   switch (dt) {
@@ -130,18 +159,21 @@ int max_partitions(int max_context_len, int partition_size) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Split-K workspace: m, l [S][Hq][NP] fp32, o [S][Hq][NP][D] fp32, then one
+// counter per (sequence, KV head); each section 256-byte aligned.
 struct WorkspaceLayout {
-  size_t m_off, l_off, o_off, bytes;
+  size_t m_off, l_off, o_off, c_off, bytes;
 };
 
-WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int np) {
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int np) {
   WorkspaceLayout w{};
   if (np <= 1) return w;
   const size_t rows = (size_t)num_seqs * num_heads * np;
   w.m_off = 0;
   w.l_off = align256(rows * sizeof(float));
   w.o_off = w.l_off + align256(rows * sizeof(float));
-  w.bytes = w.o_off + align256(rows * head_dim * sizeof(float));
+  w.c_off = w.o_off + align256(rows * head_dim * sizeof(float));
+  w.bytes = w.c_off + align256((size_t)num_seqs * num_kv_heads * sizeof(unsigned));
   return w;
 }
 
@@ -156,12 +188,18 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
   const long long grid = (long long)p.num_seqs * p.num_kv_heads * p.max_partitions;
   if (grid == 0) return PA_OK;
   if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  if (p.ws_count != nullptr) {   // split call, combined in the partition kernel: counters start at 0
+    const int n = p.num_seqs * p.num_kv_heads;
+    const int ctas = (n + 255) / 256 < sm_count() ? (n + 255) / 256 : sm_count();
+    pa_status_t st = launch(pa::zero_counts_kernel, dim3((unsigned)ctas), dim3(256), 0, stream, p.ws_count, n);
+    if (st != PA_OK) return st;
+  }
   pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(pa::kDecodeThreads), SM::kAlloc, stream, mk, mv, p);
-  if (st != PA_OK || p.max_partitions <= 1) return st;
+  if (st != PA_OK || p.max_partitions <= 1 || p.ws_count != nullptr) return st;
   // a fixed grid of warps walks all (sequence, head) rows: 8 CTAs of 4 warps per SM at most
   const long long rows = (long long)p.num_seqs * p.num_heads;
   long long ctas = (rows + pa::kReduceWarps - 1) / pa::kReduceWarps;
-  if (ctas > 148LL * 8) ctas = 148LL * 8;
+  if (ctas > 8LL * sm_count()) ctas = 8LL * sm_count();
   return launch(pa::pa_decode_reduce_kernel<T>, dim3((unsigned)ctas), dim3(pa::kReduceWarps * 32), 0, stream, p);
 }
 
@@ -218,7 +256,7 @@ pa_status_t pa_reshape_and_cache(const void *key, const void *value, void *k_cac
   const int chunks_per_slot = num_kv_heads * (row_bytes(dtype) / 16);
   const long long total = (long long)num_tokens * chunks_per_slot;
   long long blocks = (total + 255) / 256;
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  if (blocks > 16LL * sm_count()) blocks = 16LL * sm_count();
   return launch(pa::reshape_and_cache_kernel, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream,
                 (const uint4 *)key, (const uint4 *)value, (uint4 *)k_cache, (uint4 *)v_cache, slot_mapping,
                 num_tokens, chunks_per_slot, (long long)num_blocks * block_size);
@@ -235,20 +273,31 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, 
   const int P = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
                                          requested_partition_size);
   if (P <= 0) return 0;
-  return workspace_layout(num_seqs, num_heads, head_dim, max_partitions(max_context_len, P)).bytes;
+  return workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_partitions(max_context_len, P)).bytes;
 }
 
 }  // extern "C"
 
 namespace {
 
-// dtype: the cache dtype; q_dtype: q and out (equal to dtype except for E4M3 caches)
-pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void *new_v, const void *k_cache,
-                        const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+// A decode call's arguments, checked, with the partition plan derived from them.
+struct DecodePlan {
+  pa::DecodeParams p;
+  CUtensorMap mk, mv;
+  const void *k_cache, *v_cache;
+  WorkspaceLayout ws;
+  int group;
+  pa_dtype_t dtype, q_dtype;
+  bool empty;   // nothing to launch (no sequences)
+};
+
+// Every host-side check of a decode call, in order, except the workspace's:
+// dtype: the cache dtype; q_dtype: q and out (equal to dtype except for E4M3 caches).
+pa_status_t plan_decode(DecodePlan &d, void *out, const void *q, const void *new_k, const void *new_v,
+                        const void *k_cache, const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                         const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len, float scale,
-                        int partition_size, void *workspace, size_t workspace_bytes, int64_t num_blocks,
-                        int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream,
-                        pa_dtype_t q_dtype, float k_scale, float v_scale) {
+                        int partition_size, int64_t num_blocks, int block_size, int num_kv_heads, int head_dim,
+                        pa_dtype_t dtype, pa_dtype_t q_dtype, float k_scale, float v_scale) {
   pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
   if (st != PA_OK) return st;
   if (dtype == PA_FP8_E4M3 ? (q_dtype != PA_F16 && q_dtype != PA_BF16) : q_dtype != dtype) return PA_ERR_DTYPE;
@@ -262,33 +311,25 @@ pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void 
   const int P = resolve_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
                                        partition_size);
   if (P <= 0) return PA_ERR_SHAPE;
-  if (num_seqs == 0) return PA_OK;
+  d.empty = num_seqs == 0;
+  if (d.empty) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !context_lens || (max_blocks_per_seq > 0 && !block_tables))
     return PA_ERR_NULL;
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
       !aligned(block_tables, 4) || !aligned(context_lens, 4))
     return PA_ERR_ALIGN;
   const int np = max_partitions(max_context_len, P);
-  const WorkspaceLayout ws = workspace_layout(num_seqs, num_heads, head_dim, np);
-  if (ws.bytes > 0) {
-    if (!workspace || workspace_bytes < ws.bytes) return PA_ERR_WORKSPACE;
-    if (!aligned(workspace, 256)) return PA_ERR_ALIGN;
-  }
+  d.ws = workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, np);
+  d.group = group;
+  d.dtype = dtype;
+  d.q_dtype = q_dtype;
 
-  CUtensorMap mk, mv;
-  if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, row_bytes(dtype)) ||
-      !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, row_bytes(dtype)))
-    return PA_ERR_CUDA;
-
-  pa::DecodeParams p{};
+  pa::DecodeParams &p = d.p;
+  p = pa::DecodeParams{};
   p.out = out;
   p.q = q;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
-  char *w = static_cast<char *>(workspace);
-  p.ws_m = ws.bytes ? reinterpret_cast<float *>(w + ws.m_off) : nullptr;
-  p.ws_l = ws.bytes ? reinterpret_cast<float *>(w + ws.l_off) : nullptr;
-  p.ws_o = ws.bytes ? reinterpret_cast<float *>(w + ws.o_off) : nullptr;
   p.num_blocks = num_blocks;
   p.num_seqs = num_seqs;
   p.num_heads = num_heads;
@@ -303,18 +344,55 @@ pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void 
   p.new_v = new_v;
   p.k_cache = new_k ? const_cast<void *>(k_cache) : nullptr;
   p.v_cache = new_k ? const_cast<void *>(v_cache) : nullptr;
+  d.k_cache = k_cache;
+  d.v_cache = v_cache;
+  return PA_OK;
+}
 
+// Launch a planned decode with its split-K workspace (checked by the caller).
+pa_status_t launch_planned(DecodePlan &d, void *workspace, void *stream) {
+  if (d.empty) return PA_OK;
+  pa::DecodeParams &p = d.p;
+  const int rb = row_bytes(d.dtype);
+  if (!encode_cache_map(&d.mk, d.k_cache, p.num_blocks, p.num_kv_heads, rb) ||
+      !encode_cache_map(&d.mv, d.v_cache, p.num_blocks, p.num_kv_heads, rb))
+    return PA_ERR_CUDA;
+  char *w = static_cast<char *>(workspace);
+  p.ws_m = d.ws.bytes ? reinterpret_cast<float *>(w + d.ws.m_off) : nullptr;
+  p.ws_l = d.ws.bytes ? reinterpret_cast<float *>(w + d.ws.l_off) : nullptr;
+  p.ws_o = d.ws.bytes ? reinterpret_cast<float *>(w + d.ws.o_off) : nullptr;
+  p.ws_count = d.ws.bytes && PA_FUSED_COMBINE ? reinterpret_cast<unsigned *>(w + d.ws.c_off) : nullptr;
+  p.stall_cta = g_stall_decode.exchange(0);
   cudaStream_t s = (cudaStream_t)stream;
-  if (dtype == PA_FP8_E4M3)
-    return q_dtype == PA_F16 ? dispatch_group_fp8<__half>(group, mk, mv, p, s)
-                             : dispatch_group_fp8<__nv_bfloat16>(group, mk, mv, p, s);
-  switch (dtype) {
-    case PA_F32: return dispatch_group<float>(group, mk, mv, p, s);
-    case PA_F16: return dispatch_group<__half>(group, mk, mv, p, s);
-    case PA_BF16: return dispatch_group<__nv_bfloat16>(group, mk, mv, p, s);
+  const int group = d.group;
+  if (d.dtype == PA_FP8_E4M3)
+    return d.q_dtype == PA_F16 ? dispatch_group_fp8<__half>(group, d.mk, d.mv, p, s)
+                               : dispatch_group_fp8<__nv_bfloat16>(group, d.mk, d.mv, p, s);
+  switch (d.dtype) {
+    case PA_F32: return dispatch_group<float>(group, d.mk, d.mv, p, s);
+    case PA_F16: return dispatch_group<__half>(group, d.mk, d.mv, p, s);
+    case PA_BF16: return dispatch_group<__nv_bfloat16>(group, d.mk, d.mv, p, s);
     case PA_FP8_E4M3: break;
   }
   return PA_ERR_DTYPE;
+}
+
+pa_status_t decode_impl(void *out, const void *q, const void *new_k, const void *new_v, const void *k_cache,
+                        const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                        const int32_t *context_lens, int num_seqs, int num_heads, int max_context_len, float scale,
+                        int partition_size, void *workspace, size_t workspace_bytes, int64_t num_blocks,
+                        int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype, void *stream,
+                        pa_dtype_t q_dtype, float k_scale, float v_scale) {
+  DecodePlan d;
+  const pa_status_t st = plan_decode(d, out, q, new_k, new_v, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                     context_lens, num_seqs, num_heads, max_context_len, scale, partition_size,
+                                     num_blocks, block_size, num_kv_heads, head_dim, dtype, q_dtype, k_scale, v_scale);
+  if (st != PA_OK || d.empty) return st;
+  if (d.ws.bytes > 0) {
+    if (!workspace || workspace_bytes < d.ws.bytes) return PA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return PA_ERR_ALIGN;
+  }
+  return launch_planned(d, workspace, stream);
 }
 
 }  // namespace
@@ -360,7 +438,7 @@ pa_status_t pa_reshape_and_cache_fp8(const void *key, const void *value, void *k
   const int chunks_per_slot = num_kv_heads * (head_dim / 8);   // 8 elements per thread
   const long long total = (long long)num_tokens * chunks_per_slot;
   long long blocks = (total + 255) / 256;
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  if (blocks > 16LL * sm_count()) blocks = 16LL * sm_count();
   const long long slots = (long long)num_blocks * block_size;
   if (src_dtype == PA_F16)
     return launch(pa::reshape_and_cache_fp8_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0,
@@ -423,6 +501,7 @@ pa_status_t pa_prefill(void *out, const void *q, const void *k_cache, const void
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.max_query_len = max_query_len;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.stall_cta = g_stall_prefill.exchange(0);
   const int qt = pa::kPrefillTiles * pa::kPrefillRows / group;   // chunk queries per CTA
   const dim3 grid((unsigned)((max_query_len + qt - 1) / qt), (unsigned)num_kv_heads, (unsigned)num_seqs);
   auto go = [&](auto kernel) -> pa_status_t {
@@ -454,13 +533,18 @@ pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_ma
                            void *stream) {
   pa_status_t st = cache_shape_status(num_blocks, block_size, num_kv_heads, head_dim, dtype);
   if (st != PA_OK) return st;
-  if (num_pairs < 0 || num_pairs > 65535 * 1024) return PA_ERR_SHAPE;
+  if (num_pairs < 0 || num_pairs > PA_MAX_COPY_PAIRS) return PA_ERR_SHAPE;
   if (num_pairs == 0) return PA_OK;
   if (!k_cache || !v_cache || !block_mapping) return PA_ERR_NULL;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8)) return PA_ERR_ALIGN;
   const int chunks_per_block = kBlockSize * num_kv_heads * (row_bytes(dtype) / 16);
-  return launch(pa::copy_blocks_kernel, dim3((unsigned)num_pairs, 2), dim3(256), 0, (cudaStream_t)stream,
-                (uint4 *)k_cache, (uint4 *)v_cache, (const long long *)block_mapping, num_pairs,
+  // one CTA per pair up to two per SM, then each CTA takes several pairs (at
+  // most kCopyMaxPairsPerCta); blockIdx.y: 0 = K cache, 1 = V cache
+  long long ctas = num_pairs < 2LL * sm_count() ? num_pairs : 2LL * sm_count();
+  const long long min_ctas = (num_pairs + pa::kCopyMaxPairsPerCta - 1) / pa::kCopyMaxPairsPerCta;
+  if (ctas < min_ctas) ctas = min_ctas;
+  return launch(pa::copy_blocks_kernel, dim3((unsigned)ctas, 2), dim3(pa::kCopyThreads), 0, (cudaStream_t)stream,
+                (uint4 *)k_cache, (uint4 *)v_cache, (const longlong2 *)block_mapping, num_pairs,
                 (long long)num_blocks, chunks_per_block);
 }
 
@@ -472,22 +556,14 @@ pa_status_t pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_ma
 static __device__ __align__(256) unsigned char g_decode_scratch[PA_STATIC_WORKSPACE_BYTES];
 
 namespace {
-constexpr int kMaxScratchDevices = 128;
-std::mutex g_scratch_mutex;
-void *g_scratch_ptr[kMaxScratchDevices] = {};
-
-// Address of this device's copy of g_decode_scratch; looked up once per device
-// (with that device current) and cached.
+// Address of the current device's copy of g_decode_scratch, looked up on every
+// call (cheap, allocates nothing), so that it is never stale -- e.g. after a
+// cudaDeviceReset, which gives the device a new context and a new copy.  The
+// first lookup on a device may load the library's device code there.
 void *scratch_for_current_device() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return nullptr;
-    g_scratch_ptr[dev] = ptr;
-  }
-  return g_scratch_ptr[dev];
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) return nullptr;
+  return ptr;
 }
 }  // namespace
 
@@ -497,17 +573,43 @@ pa_status_t pa_decode_static_workspace(void *out, const void *q, const void *k_c
                                        int max_context_len, float scale, int partition_size, int64_t num_blocks,
                                        int block_size, int num_kv_heads, int head_dim, pa_dtype_t dtype,
                                        void *stream) {
-  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_SHAPE;
-  const int P = resolve_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
-                                       partition_size);
-  if (P <= 0) return PA_ERR_SHAPE;
-  const size_t need = workspace_layout(num_seqs, num_heads, head_dim, max_partitions(max_context_len, P)).bytes;
-  if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_WORKSPACE;
-  void *scratch = scratch_for_current_device();
-  if (!scratch) return PA_ERR_CUDA;
-  return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_heads,
-                   max_context_len, scale, partition_size, scratch, PA_STATIC_WORKSPACE_BYTES, num_blocks,
-                   block_size, num_kv_heads, head_dim, dtype, stream);
+  if (dtype == PA_FP8_E4M3) return PA_ERR_DTYPE;   // as pa_decode
+  // every check of pa_decode first, in its order; then the size of the scratch
+  DecodePlan d;
+  const pa_status_t st = plan_decode(d, out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                     context_lens, num_seqs, num_heads, max_context_len, scale, partition_size,
+                                     num_blocks, block_size, num_kv_heads, head_dim, dtype, dtype, 1.f, 1.f);
+  if (st != PA_OK || d.empty) return st;
+  void *scratch = nullptr;
+  if (d.ws.bytes > 0) {
+    if (d.ws.bytes > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_WORKSPACE;
+    scratch = scratch_for_current_device();
+    if (!scratch) return PA_ERR_CUDA;
+  }
+  return launch_planned(d, scratch, stream);
+}
+
+pa_status_t pa_stream_read(const void *buf, size_t bytes, uint64_t *sink, void *stream) {
+  if (bytes % 16 != 0) return PA_ERR_SHAPE;
+  if (bytes == 0) return PA_OK;
+  if (!buf || !sink) return PA_ERR_NULL;
+  if (!aligned(buf, 16) || !aligned(sink, 8)) return PA_ERR_ALIGN;
+  // eight resident CTAs of 256 threads per SM: a full SM of threads
+  const long long n16 = (long long)(bytes / 16);
+  long long ctas = (n16 + pa::kProbeThreads - 1) / pa::kProbeThreads;
+  if (ctas > 8LL * sm_count()) ctas = 8LL * sm_count();
+  return launch(pa::stream_read_kernel, dim3((unsigned)ctas), dim3(pa::kProbeThreads), 0, (cudaStream_t)stream,
+                (const uint4 *)buf, n16, (unsigned long long *)sink);
+}
+
+pa_status_t pa_test_stall_next_launch(int kernel, int64_t cta) {
+  if (cta < -1 || cta >= INT32_MAX) return PA_ERR_SHAPE;
+  const int armed = (int)cta + 1;   // cta -1: disarm
+  switch (kernel) {
+    case 0: g_stall_decode.store(armed); return PA_OK;
+    case 1: g_stall_prefill.store(armed); return PA_OK;
+  }
+  return PA_ERR_SHAPE;
 }
 
 int pa_get_device_error(void *stream, int64_t *detail, int clear) {

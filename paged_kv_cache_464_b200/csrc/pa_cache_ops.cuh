@@ -88,35 +88,69 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(const uint4 
 }
 
 // Copy-on-write block copy ("vLLM 原理与源码阅读", Block 管理器, item 3).
-// blockIdx.x = pair, blockIdx.y = 0 for the K cache, 1 for the V cache.
-// Every CTA first checks its pair against all pairs (conflicting pairs are
-// skipped, as are out-of-range ids), then copies one whole block.
-__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
-                                                          const long long *__restrict__ block_mapping,
-                                                          int num_pairs, long long num_blocks,
-                                                          int chunks_per_block) {
+// blockIdx.y = 0 for the K cache, 1 for the V cache; CTA x takes the pairs
+// x, x + gridDim.x, ... (at most kCopyMaxPairsPerCta of them).  A pair is
+// skipped when an id is out of range or when its dst is the dst of another pair
+// or the src of any pair (the set of pairs decides, not their order).  The
+// check streams all pairs once through shared memory in chunks of
+// kCopyChunkPairs and compares them with this CTA's own pairs there: each CTA
+// reads the mapping once (num_pairs x 16 bytes, from L2) and does
+// (its pairs) x num_pairs comparisons in shared memory, so the whole check is
+// num_pairs^2 shared-memory comparisons and gridDim x num_pairs x 16 bytes of
+// reads.  Then each CTA copies its non-skipped blocks.
+constexpr int kCopyThreads = 256;
+constexpr int kCopyChunkPairs = 1024;      // pairs staged in shared memory at a time (16 KiB)
+constexpr int kCopyMaxPairsPerCta = 256;   // with PA_MAX_COPY_PAIRS = 65536: at least 256 CTAs
+
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(uint4 *__restrict__ k_cache,
+                                                                   uint4 *__restrict__ v_cache,
+                                                                   const longlong2 *__restrict__ block_mapping,
+                                                                   int num_pairs, long long num_blocks,
+                                                                   int chunks_per_block) {
+  __shared__ longlong2 chunk[kCopyChunkPairs];
+  __shared__ long long mine_dst[kCopyMaxPairsPerCta];
+  __shared__ int mine_bad[kCopyMaxPairsPerCta];    // an id out of range
+  __shared__ int mine_conf[kCopyMaxPairsPerCta];   // dst repeated or read by a pair
   pdl_wait();
   pdl_trigger();
-  const int pair = blockIdx.x;
-  const long long src = block_mapping[2 * pair];
-  const long long dst = block_mapping[2 * pair + 1];
-  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
-    if (threadIdx.x == 0 && blockIdx.y == 0) record_error(1 /*PA_DEV_BAD_BLOCK_ID*/, src < 0 || src >= num_blocks ? src : dst);
-    return;
+  const int n_mine = (num_pairs - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1;
+  for (int m = threadIdx.x; m < n_mine; m += kCopyThreads) {
+    const longlong2 pr = block_mapping[blockIdx.x + static_cast<long long>(m) * gridDim.x];
+    const bool bad = pr.x < 0 || pr.x >= num_blocks || pr.y < 0 || pr.y >= num_blocks;
+    mine_dst[m] = pr.y;
+    mine_bad[m] = bad ? 1 : 0;
+    mine_conf[m] = 0;
+    if (bad && blockIdx.y == 0) record_error(1 /*PA_DEV_BAD_BLOCK_ID*/, pr.x < 0 || pr.x >= num_blocks ? pr.x : pr.y);
   }
-  int conflict = 0;
-  for (int j = threadIdx.x; j < num_pairs; j += blockDim.x) {
-    const long long sj = block_mapping[2 * j], dj = block_mapping[2 * j + 1];
-    conflict |= (j != pair && dj == dst) || sj == dst;
+  for (int c0 = 0; c0 < num_pairs; c0 += kCopyChunkPairs) {
+    const int n = min(kCopyChunkPairs, num_pairs - c0);
+    __syncthreads();   // the previous chunk's comparisons are done (and mine_* are written)
+    for (int e = threadIdx.x; e < n; e += kCopyThreads) chunk[e] = block_mapping[c0 + e];
+    __syncthreads();
+    for (int e = threadIdx.x; e < n; e += kCopyThreads) {
+      const long long src = chunk[e].x, dst = chunk[e].y;
+      const int pair_e = c0 + e;
+      for (int m = 0; m < n_mine; ++m) {
+        const long long d = mine_dst[m];
+        const int pair_m = static_cast<int>(blockIdx.x) + m * static_cast<int>(gridDim.x);
+        if (src == d || (dst == d && pair_e != pair_m)) mine_conf[m] = 1;   // every writer writes 1
+      }
+    }
   }
-  if (__syncthreads_or(conflict)) {
-    if (threadIdx.x == 0 && blockIdx.y == 0) record_error(3 /*PA_DEV_COPY_CONFLICT*/, pair);
-    return;
-  }
+  __syncthreads();
   uint4 *cache = blockIdx.y == 0 ? k_cache : v_cache;
-  const uint4 *s = cache + src * chunks_per_block;
-  uint4 *d = cache + dst * chunks_per_block;
-  for (int i = threadIdx.x; i < chunks_per_block; i += blockDim.x) d[i] = s[i];
+  for (int m = 0; m < n_mine; ++m) {
+    const long long pair = blockIdx.x + static_cast<long long>(m) * gridDim.x;
+    if (mine_bad[m]) continue;   // recorded above
+    if (mine_conf[m]) {
+      if (threadIdx.x == 0 && blockIdx.y == 0) record_error(3 /*PA_DEV_COPY_CONFLICT*/, pair);
+      continue;
+    }
+    const longlong2 pr = block_mapping[pair];
+    const uint4 *s = cache + pr.x * chunks_per_block;
+    uint4 *d = cache + pr.y * chunks_per_block;
+    for (int i = threadIdx.x; i < chunks_per_block; i += kCopyThreads) d[i] = s[i];
+  }
 }
 
 }  // namespace pa

@@ -70,14 +70,29 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// Wait for phase `parity` of `bar` to complete; false if it has not after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Wait for phase `parity` of `bar` to complete; false if it has not after
+// `limit_ns` (kWaitLimitNs unless a test shortens it for one CTA).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+    if ((it & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Test hook for the bounded-wait error path.  A kernel launched with
+// stall_cta = c + 1 (0 = off, the value of every ordinary launch) treats its CTA
+// c specially: that CTA leaves one of its copies unissued -- no copy and no
+// barrier arrival, so nothing is in flight for that stage -- and its waits give
+// up after kTestWaitLimitNs instead of kWaitLimitNs.  The wait on the missing
+// stage therefore runs out, and the CTA takes the same abort path a real
+// timeout would.  Every other CTA runs as usual.
+constexpr unsigned long long kTestWaitLimitNs = 1000000ull;   // 1 ms
+
+__device__ __forceinline__ unsigned long long wait_limit_for(int stall_cta, long long cta) {
+  return stall_cta != 0 && cta == stall_cta - 1 ? kTestWaitLimitNs : kWaitLimitNs;
 }
 
 // ---------------------------------------------------------------- TMA

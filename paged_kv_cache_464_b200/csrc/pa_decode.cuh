@@ -76,6 +76,7 @@ struct DecodeParams {
   float *ws_m;                    // [S][Hq][NPmax]
   float *ws_l;                    // [S][Hq][NPmax]
   float *ws_o;                    // [S][Hq][NPmax][D]
+  unsigned *ws_count;             // [S][Hkv] partitions done (zeroed before the launch); null: separate reduce
   long long num_blocks;
   int num_seqs, num_heads, num_kv_heads, max_blocks_per_seq;
   int max_context_len, partition_size, max_partitions;
@@ -85,6 +86,7 @@ struct DecodeParams {
   // rows [S][Hkv][D], written at position context_len - 1 before it is attended
   const void *new_k, *new_v;
   void *k_cache, *v_cache;
+  int stall_cta;                  // test hook (pa_common.cuh): 0 in every ordinary launch
 };
 
 // Byte offset of 16-byte chunk `c` (0..15) of token `t` in a swizzled tile.
@@ -636,11 +638,86 @@ struct DecodeSmem {
   static constexpr int kMOff = kScratchOff + Math::kScratchBytes;
   static constexpr int kLOff = kMOff + kDecodeWarps * G * 4;
   static constexpr int kFlagOff = kLOff + kDecodeWarps * G * 4;
-  static constexpr int kBarOff = (kFlagOff + 4 + 7) / 8 * 8;
+  static constexpr int kBarOff = (kFlagOff + 8 + 7) / 8 * 8;   // abort flag, last-partition flag
   static constexpr int kBytes = kBarOff + kStages * 8;
   static constexpr int kAlloc = kBytes + 1024;   // room to align the base to 1024 B (128B swizzle atom)
   static_assert(kDecodeWarps * G * D * 4 <= kTilesBytes, "epilogue buffer must fit in the stage tiles");
 };
+
+// ============================================================ split-K combine
+// out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p over the nparts partials of
+// the G heads h0 .. h0+G-1 of sequence b (M = max_p m_p; m_p base-2 maxima, o_p
+// and l_p relative to m_p).  Run by one CTA of the partition kernel, the last
+// to finish for that (sequence, KV head).  Same arithmetic, in the same order,
+// as pa_decode_reduce_kernel: per head, lane-strided max and sum over the
+// partitions joined by shuffles, then o accumulated over the partitions in
+// order.  Partials are read through L2 (.cg): other SMs wrote them.
+template <typename T, int G, int D>
+__device__ __forceinline__ void combine_partitions(const DecodeParams &p, int b, int h0, int nparts, float *M_s,
+                                                   float *inv_s, T *out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int hh = warp; hh < G; hh += kDecodeWarps) {
+    const size_t row = static_cast<size_t>(b) * p.num_heads + h0 + hh;
+    const float *m = p.ws_m + row * p.max_partitions;
+    const float *l = p.ws_l + row * p.max_partitions;
+    float M = -INFINITY;
+    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, __ldcg(m + i));
+    M = warp_max(M);
+    float lsum = 0.f;
+    for (int i = lane; i < nparts; i += 32) lsum += ex2(__ldcg(m + i) - M) * __ldcg(l + i);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, off);
+    if (lane == 0) {
+      M_s[hh] = M;
+      inv_s[hh] = 1.f / lsum;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x * 4; i < G * D; i += kDecodeThreads * 4) {
+    const int hh = i / D, d = i % D;
+    const size_t row = static_cast<size_t>(b) * p.num_heads + h0 + hh;
+    const float *m = p.ws_m + row * p.max_partitions;
+    const float *o = p.ws_o + row * p.max_partitions * D + d;
+    const float M = M_s[hh];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int k = 0;
+    for (; k + 8 <= nparts; k += 8) {   // eight partials in flight
+      float w[8];
+      float4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        w[u] = __ldcg(m + k + u);
+        x[u] = __ldcg(reinterpret_cast<const float4 *>(o + static_cast<size_t>(k + u) * D));
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float wk = ex2(w[u] - M);
+        acc.x += wk * x[u].x;
+        acc.y += wk * x[u].y;
+        acc.z += wk * x[u].z;
+        acc.w += wk * x[u].w;
+      }
+    }
+    for (; k < nparts; ++k) {
+      const float wk = ex2(__ldcg(m + k) - M);
+      const float4 x = __ldcg(reinterpret_cast<const float4 *>(o + static_cast<size_t>(k) * D));
+      acc.x += wk * x.x;
+      acc.y += wk * x.y;
+      acc.z += wk * x.z;
+      acc.w += wk * x.w;
+    }
+    const float inv = inv_s[hh];
+    Elem<T>::store4(out + i, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+}
+
+// Zero the per-(sequence, KV head) partition counters of a split call; launched
+// (programmatically) just before the partition kernel of the same call.
+__global__ void __launch_bounds__(256) zero_counts_kernel(unsigned *count, int n) {
+  pdl_wait();   // the previous kernel in the stream (which may use the same workspace) is done
+  pdl_trigger();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) count[i] = 0u;
+}
 
 // ============================================================ partition kernel
 template <typename T, int G, typename Math>
@@ -659,10 +736,13 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   float *m_s = reinterpret_cast<float *>(smem + SM::kMOff);
   float *l_s = reinterpret_cast<float *>(smem + SM::kLOff);
   int *abort_s = reinterpret_cast<int *>(smem + SM::kFlagOff);
+  int *last_s = abort_s + 1;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::kBarOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const unsigned long long wait_limit = wait_limit_for(p.stall_cta, blockIdx.x);
+  const bool stall_here = p.stall_cta != 0 && static_cast<int>(blockIdx.x) == p.stall_cta - 1;
   pdl_wait();      // the previous kernel's writes (caches, inputs) are visible from here on
   pdl_trigger();   // the reduce kernel may be scheduled once every CTA of this grid has started
 
@@ -720,7 +800,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
     }
     const int id = __shfl_sync(kFullMask, my_id, j & 31);
     const int s = warp + (j % kSPW) * kDecodeWarps;
-    if (lane == 0) {
+    if (lane == 0 && !(stall_here && warp == 0 && j == 0)) {   // (test hook: warp 0's first stage left unissued)
       if (id >= 0) {
         // one box per 128-byte part of the rows: the tile lands as [part][token][128 B]
         uint8_t *tk = smem + s * 2 * kTile;
@@ -748,7 +828,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   int j = 0;
   for (; j < nw; ++j) {
     const int s = warp + (j % kSPW) * kDecodeWarps;
-    const bool landed = mbar_wait(&full[s], (j / kSPW) & 1);
+    const bool landed = mbar_wait(&full[s], (j / kSPW) & 1, wait_limit);
     if (!__all_sync(kFullMask, landed)) {
       if (lane == 0) {
         record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, blockIdx.x);
@@ -788,9 +868,11 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
     }
   }
   if (!ok) {
-    // let this warp's other copies in flight land (bounded) before the CTA can exit
-    for (int jj = j + 1; jj < min(nw, j + kSPW); ++jj)
-      mbar_wait(&full[warp + (jj % kSPW) * kDecodeWarps], (jj / kSPW) & 1);
+    // let this warp's copies in flight land (bounded) before the CTA can exit:
+    // the stages of blocks j .. j + kSPW - 1, the one that timed out included
+    // (its copy may still arrive)
+    for (int jj = j; jj < min(nw, j + kSPW); ++jj)
+      mbar_wait(&full[warp + (jj % kSPW) * kDecodeWarps], (jj / kSPW) & 1, wait_limit);
   }
 
   // ---- merge the warps through shared memory (the stage tiles are reused)
@@ -829,6 +911,19 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
       }
     }
   }
+  if (nparts == 1 || p.ws_count == nullptr) return;
+
+  // ---- split sequence: the last of its nparts CTAs (per KV head) combines the
+  // partials.  Publish this CTA's partial, then take a ticket; no CTA waits for
+  // another, and the ticket that completes the count goes to exactly one CTA.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    *last_s = atomicAdd(p.ws_count + static_cast<size_t>(b) * p.num_kv_heads + g, 1u) == static_cast<unsigned>(nparts - 1);
+  __syncthreads();
+  if (!*last_s) return;
+  __threadfence();   // the other CTAs' partials (published before their tickets) are visible from here on
+  combine_partitions<T, G, D>(p, b, h0, nparts, m_s, l_s, out);
 }
 
 // Combine the partitions of every (sequence, query head) that was split:

@@ -62,6 +62,7 @@ struct PrefillParams {
   long long num_blocks;
   int num_seqs, num_heads, num_kv_heads, max_blocks_per_seq, max_query_len;
   float scale_log2;                   // scale * log2(e), > 0
+  int stall_cta;                      // test hook (pa_common.cuh): 0 in every ordinary launch
 };
 
 constexpr int kPrefillRows = 128;        // M: rows of one query tile
@@ -167,17 +168,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
-// Bounded wait that also gives up once another role has raised the abort flag.
-// With `backoff` the waiting warp sleeps between polls, leaving the shared
-// memory ports (which also feed the tensor cores' operands) to others.
+// Bounded wait (`limit_ns`) that also gives up once another role has raised
+// the abort flag.  With `backoff` the waiting warp sleeps between polls,
+// leaving the shared memory ports (which also feed the tensor cores' operands)
+// to others.
 __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, const volatile int *abort_flag,
-                                                   bool backoff = false) {
+                                                   unsigned long long limit_ns, bool backoff = false) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (backoff) __nanosleep(64);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && (*abort_flag || global_ns() - t0 > kWaitLimitNs)) return false;
+    if ((it & 63u) == 0 && (*abort_flag || global_ns() - t0 > limit_ns)) return false;
   }
 }
 
@@ -209,6 +211,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  // linear CTA index: reported with PA_DEV_WAIT_TIMEOUT, and the test hook's key
+  const long long cta = blockIdx.x + static_cast<long long>(gridDim.x) * (blockIdx.y + static_cast<long long>(gridDim.y) * blockIdx.z);
+  const unsigned long long wait_limit = wait_limit_for(p.stall_cta, cta);
+  const bool stall_here = p.stall_cta != 0 && cta == p.stall_cta - 1;
   pdl_wait();
   pdl_trigger();
 
@@ -330,7 +336,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int ids[4];
 #pragma unroll
       for (int bi = 0; bi < 4; ++bi) ids[bi] = __shfl_sync(kFullMask, my_id, (4 * j + bi) & 31);
-      if (lane == 0) {
+      const bool skip = stall_here && j == 0 && !is_v;   // test hook: K tile 0 left unissued
+      if (lane == 0 && !skip) {
         const int st = j % (is_v ? VS : KS);
         uint8_t *dst = smem + (is_v ? SM::kV : SM::kK) + st * SM::kKvTileBytes;
         uint64_t *bar = is_v ? &v_full[st] : &k_full[st];
@@ -343,12 +350,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         ids[bi], bar);
       }
       if (is_v) last_v[j % VS] = j;
-      else last_k[j % KS] = j;
+      else if (!skip) last_k[j % KS] = j;
     };
     for (int j = 0; j < ntiles; ++j) {
-      if (j >= KS && !__all_sync(kFullMask, mbar_wait_or_abort(&k_free[j % KS], (j / KS - 1) & 1, abort_s, true))) break;
+      if (j >= KS &&
+          !__all_sync(kFullMask, mbar_wait_or_abort(&k_free[j % KS], (j / KS - 1) & 1, abort_s, wait_limit, true)))
+        break;
       issue(j, false);
-      if (j >= VS && !__all_sync(kFullMask, mbar_wait_or_abort(&v_free[j % VS], (j / VS - 1) & 1, abort_s, true))) break;
+      if (j >= VS &&
+          !__all_sync(kFullMask, mbar_wait_or_abort(&v_free[j % VS], (j / VS - 1) & 1, abort_s, wait_limit, true)))
+        break;
       issue(j, true);
     }
   } else if ((warp == kPrefillMmaWarp || warp == kPrefillMmaWarp + 2) && lane == 0) {
@@ -364,9 +375,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     bool ok = true;
     auto wait = [&](uint64_t *bar, uint32_t parity) {
       if (!ok) return;
-      ok = mbar_test_wait(bar, parity) || mbar_wait_or_abort(bar, parity, abort_s);
+      ok = mbar_test_wait(bar, parity) || mbar_wait_or_abort(bar, parity, abort_s, wait_limit);
       if (!ok) {
-        record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, blockIdx.x);
+        record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, cta);
         *abort_s = 1;
       }
       tc_fence_after();
@@ -474,9 +485,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     bool ok = true;
     auto wait = [&](uint64_t *bar, uint32_t parity) {
       if (!ok) return;
-      ok = __all_sync(kFullMask, mbar_wait_or_abort(bar, parity, abort_s, true));
+      ok = __all_sync(kFullMask, mbar_wait_or_abort(bar, parity, abort_s, wait_limit, true));
       if (!ok && lane == 0) {
-        record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, blockIdx.x);
+        record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, cta);
         *abort_s = 1;
       }
       tc_fence_after();
@@ -572,14 +583,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   __syncthreads();
   if ((warp == kPrefillMmaWarp || warp == kPrefillMmaWarp + 2) && lane == 0) {
     umma_commit(drain);   // both issuers: their own operations (and commit arrivals) complete
-    mbar_wait(drain, 0);
+    mbar_wait(drain, 0, wait_limit);
   }
   if (*abort_s && warp == kPrefillLoadWarp && lane == 0) {
     // every stage: the last tile issued into it (its earlier phases completed before it was reissued)
     for (int i = 0; i < KS; ++i)
-      if (last_k[i] >= 0) mbar_wait(&k_full[i], (last_k[i] / KS) & 1);
+      if (last_k[i] >= 0) mbar_wait(&k_full[i], (last_k[i] / KS) & 1, wait_limit);
     for (int i = 0; i < VS; ++i)
-      if (last_v[i] >= 0) mbar_wait(&v_full[i], (last_v[i] / VS) & 1);
+      if (last_v[i] >= 0) mbar_wait(&v_full[i], (last_v[i] / VS) & 1, wait_limit);
   }
   __syncthreads();
   if (warp == kPrefillMmaWarp) {

@@ -157,3 +157,45 @@ def test_prefill_host_validation(capi):
     assert pf(scale=float("nan")) == 3
     assert pf(qsl=None) == 1 and pf(q=None) == 1
     assert pf(out=8) == 6 and pf(qsl=2) == 6
+
+
+def test_copy_blocks_pair_cap(capi):
+    r = capi.raw
+    assert capi.MAX_COPY_PAIRS == 65536
+    assert r.pa_copy_blocks(16, 16, 16, capi.MAX_COPY_PAIRS + 1, 8, 16, 4, 64, 0, None) == 3
+
+
+def test_static_workspace_checks_follow_pa_decode(capi):
+    """pa_decode_static_workspace runs every pa_decode check first, in its order;
+    only then does an oversized scratch need return PA_ERR_WORKSPACE."""
+    r = capi.raw
+
+    def sw(**k):
+        a = dict(out=16, q=16, S=4096, maxL=32768, P=16, dt=2, D=128, Hq=64)
+        a.update(k)
+        return r.pa_decode_static_workspace(a["out"], a["q"], 16, 16, 16, 2048, 16, a["S"], a["Hq"], a["maxL"],
+                                            0.088, a["P"], 1 << 20, 16, 8, a["D"], a["dt"], None)
+    assert sw() == 4                 # too large for the library's scratch
+    assert sw(out=8) == 6            # misaligned out: pa_decode's PA_ERR_ALIGN comes first
+    assert sw(q=None) == 1           # NULL q: PA_ERR_NULL comes first
+    assert sw(dt=3) == 2             # 1-byte caches: PA_ERR_DTYPE, as pa_decode
+    assert sw(D=64) == 3             # bf16 rows must be 256 bytes
+    assert sw(P=24) == 3             # partition not a multiple of 16
+    assert sw(S=0) == 0              # nothing to do
+
+
+def test_stall_hook_arguments(capi):
+    r = capi.raw
+    assert r.pa_test_stall_next_launch(2, 0) == 3      # unknown kernel
+    assert r.pa_test_stall_next_launch(0, -2) == 3     # bad CTA index
+    assert r.pa_test_stall_next_launch(0, -1) == 0     # disarm
+    assert r.pa_test_stall_next_launch(1, -1) == 0
+
+
+def test_stream_read_host_validation(capi):
+    r = capi.raw
+    assert r.pa_stream_read(16, 0, 16, None) == 0       # nothing to read
+    assert r.pa_stream_read(16, 24, 16, None) == 3      # not a multiple of 16 bytes
+    assert r.pa_stream_read(None, 32, 16, None) == 1
+    assert r.pa_stream_read(8, 32, 16, None) == 6       # buffer not 16-byte aligned
+    assert r.pa_stream_read(16, 32, 12, None) == 6      # sink not 8-byte aligned

@@ -141,14 +141,14 @@ def test_prefill_garbage_table_tail(pa, orc):
     _no_device_error(pa)
 
 
-def test_prefill_full_size_sampled(pa, orc):
+def test_prefill_full_size_all_sequences(pa, orc):
     """The Llama-3-8B-shaped chunked-prefill workload in the launch the bench
-    times; the oracle checks four whole sequences of it."""
+    times; the oracle checks every query row of all 16 sequences."""
     case = _poison(inputs.make_prefill_case("llama3_8b_prefill"))
     out = _gpu(pa, case).cpu()
     _no_device_error(pa)
     qsl = case.query_start_loc
-    for b in (0, 5, 11, case.cfg.num_seqs - 1):
+    for b in range(case.cfg.num_seqs):
         sub = inputs.prefill_subcase(case, [b])
         ref = _ref(orc, sub)
         _close(out[int(qsl[b]):int(qsl[b + 1])], ref, f"full size, sequence {b}")

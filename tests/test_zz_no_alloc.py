@@ -5,9 +5,11 @@ device).  Its split-K scratch is the library's own fixed device array.
 
 The GPU test calls it through the C ABI twice in a row (two different
 workloads, both split into partitions so the scratch is used) and checks each
-output against pa_decode with a caller-allocated workspace, within the decode
-tolerance used everywhere else.  It needs nothing from other test files, so
-it passes alone in a fresh process as well as after the rest of the suite.
+output against pa_decode with a caller-allocated workspace: both run the same
+kernels on the same inputs, so the outputs must be bit-identical (and both are
+within the decode tolerance of the fp64 oracle, which the parity tests check).
+It needs nothing from other test files, so it passes alone in a fresh process
+as well as after the rest of the suite.
 """
 import numpy as np
 import pytest
@@ -33,7 +35,8 @@ def test_oversized_request_is_rejected_before_any_launch():
     from paged_kv_cache_464_b200 import capi
     need = capi.decode_workspace_bytes(4096, 64, 8, 128, 32768, 16)
     assert need > capi.STATIC_WORKSPACE_BYTES
-    # rejected by the size check alone: no device pointer is touched (16 is never dereferenced)
+    # every argument valid for pa_decode, only the scratch need too large: rejected
+    # before any launch (16 is a dummy, never dereferenced, device address)
     rc = capi.raw.pa_decode_static_workspace(16, 16, 16, 16, 16, 2048, 16, 4096, 64, 32768, 0.088, 16, 1 << 20,
                                              16, 8, 128, 2, None)
     assert rc == PA_ERR_WORKSPACE
@@ -66,5 +69,6 @@ def test_static_workspace_matches_caller_workspace_twice_in_a_row():
         assert rc == 0, capi.raw.pa_status_string(rc)
         torch.cuda.synchronize()
         _close(out, ref, cfg.dtype)
+        assert torch.equal(out, ref), f"{name}: differs from pa_decode with a caller workspace"
     code, detail = capi.get_device_error(clear=True)
     assert code == 0, (code, detail)
