@@ -23,7 +23,7 @@ from paged_kv_cache_464_b200 import inputs
 pytestmark = [pytest.mark.gpu, pytest.mark.expects_device_error]
 
 PA_DEV_WAIT_TIMEOUT = 5
-SENTINEL = 12345.0   # exactly representable in bf16
+SENTINEL = 12288.0   # 3 * 2^12: exactly representable in bf16 and fp16
 
 
 @pytest.fixture(scope="module")
