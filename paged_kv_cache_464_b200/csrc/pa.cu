@@ -199,11 +199,17 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
   }
   pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(pa::kDecodeThreads), SM::kAlloc, stream, mk, mv, p);
   if (st != PA_OK || p.max_partitions <= 1 || p.ws_count != nullptr) return st;
-  // a fixed grid of warps walks all (sequence, head) rows: 8 CTAs of 4 warps per SM at most
+  // warps per row: one per 8 partitions (at most kReduceWarps); a CTA takes
+  // kReduceWarps / wpr rows at a time, the grid strides over the rest (at most
+  // 8 CTAs of 8 warps per SM)
+  int wpr = (p.max_partitions + pa::kReduceBatch - 1) / pa::kReduceBatch;
+  wpr = wpr >= 8 ? 8 : wpr >= 4 ? 4 : wpr >= 2 ? 2 : 1;
   const long long rows = (long long)p.num_seqs * p.num_heads;
-  long long ctas = (rows + pa::kReduceWarps - 1) / pa::kReduceWarps;
+  const int rows_per_cta = pa::kReduceWarps / wpr;
+  long long ctas = (rows + rows_per_cta - 1) / rows_per_cta;
   if (ctas > 8LL * sm_count()) ctas = 8LL * sm_count();
-  return launch(pa::pa_decode_reduce_kernel<T>, dim3((unsigned)ctas), dim3(pa::kReduceWarps * 32), 0, stream, p);
+  return launch(pa::pa_decode_reduce_kernel<T>, dim3((unsigned)ctas), dim3(pa::kReduceWarps * 32), 0, stream, p,
+                wpr);
 }
 
 // fp32 caches and single-head groups run on the CUDA cores; 16-bit caches with

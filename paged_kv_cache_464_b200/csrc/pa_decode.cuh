@@ -648,10 +648,11 @@ struct DecodeSmem {
 // out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p over the nparts partials of
 // the G heads h0 .. h0+G-1 of sequence b (M = max_p m_p; m_p base-2 maxima, o_p
 // and l_p relative to m_p).  Run by one CTA of the partition kernel, the last
-// to finish for that (sequence, KV head).  Same arithmetic, in the same order,
-// as pa_decode_reduce_kernel: per head, lane-strided max and sum over the
-// partitions joined by shuffles, then o accumulated over the partitions in
-// order.  Partials are read through L2 (.cg): other SMs wrote them.
+// to finish for that (sequence, KV head).  Same arithmetic as
+// pa_decode_reduce_kernel (the summation order differs): per head, a
+// lane-strided max and sum over the partitions joined by shuffles, then o
+// accumulated over the partitions in order.  Partials are read through L2
+// (.cg): other SMs wrote them.
 template <typename T, int G, int D>
 __device__ __forceinline__ void combine_partitions(const DecodeParams &p, int b, int h0, int nparts, float *M_s,
                                                    float *inv_s, T *out) {
@@ -929,49 +930,66 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
 // Combine the partitions of every (sequence, query head) that was split:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
 // (m_p are base-2 log-domain maxima; o_p and l_p are relative to m_p).
-// A fixed grid of warps walks the (b, h) rows (rows that were not split are
-// skipped after one load); lane l owns outputs [l*D/32, (l+1)*D/32), so each
-// partition's partial vector is one coalesced row read.
-constexpr int kReduceWarps = 4;
+// A CTA of kReduceWarps warps takes kReduceWarps / wpr rows at a time (grid
+// stride); the wpr warps of a row split its partitions (warp k takes k, k + wpr,
+// ...), each with all of its partials' loads in flight, and join their sums
+// through shared memory.  wpr grows with the number of partitions (the host
+// picks it), so a row of 64 partials is read by 8 warps at once instead of one.
+// Lane l owns outputs [l*D/32, (l+1)*D/32): each partial vector is one
+// coalesced row read.
+constexpr int kReduceWarps = 8;
+constexpr int kReduceBatch = 8;   // partials in flight per warp
 
 template <typename T>
-__global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(const DecodeParams p, int wpr) {
   constexpr int D = kChunksPerRow * Elem<T>::kPerChunk;
   constexpr int PER_LANE = D / 32;
+  __shared__ float acc_s[kReduceWarps][D];
+  __shared__ float l_s[kReduceWarps];
   pdl_wait();   // the partition kernel's partials are visible from here on
   pdl_trigger();
-  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows_per_cta = kReduceWarps / wpr;
+  const int sub = warp % wpr;    // this warp's share of the row's partitions
+  const int rloc = warp / wpr;   // which of the CTA's rows
   const long long rows = static_cast<long long>(p.num_seqs) * p.num_heads;
-  const long long stride = static_cast<long long>(gridDim.x) * kReduceWarps;
-  for (long long row = static_cast<long long>(blockIdx.x) * kReduceWarps + (threadIdx.x >> 5); row < rows;
-       row += stride) {
-    const int b = static_cast<int>(row / p.num_heads);
-    const int L = p.context_lens[b];
-    if (L < 0 || L > p.max_context_len || L > p.max_blocks_per_seq * kBlockSize) continue;
-    const int np = (L + p.partition_size - 1) / p.partition_size;
-    if (np <= 1) continue;   // finished by the partition kernel
-    const float *m = p.ws_m + row * p.max_partitions;
-    const float *l = p.ws_l + row * p.max_partitions;
-    const float *o = p.ws_o + row * p.max_partitions * D + lane * PER_LANE;
-
-    float M = -INFINITY;
-    for (int i = lane; i < np; i += 32) M = fmaxf(M, m[i]);
-    M = warp_max(M);
+  for (long long row0 = static_cast<long long>(blockIdx.x) * rows_per_cta; row0 < rows;
+       row0 += static_cast<long long>(gridDim.x) * rows_per_cta) {   // CTA-uniform
+    const long long row = row0 + rloc;
+    int np = 0;
+    if (row < rows) {
+      const int b = static_cast<int>(row / p.num_heads);
+      const int L = p.context_lens[b];
+      if (L >= 0 && L <= p.max_context_len && L <= p.max_blocks_per_seq * kBlockSize)
+        np = (L + p.partition_size - 1) / p.partition_size;
+    }
+    const bool split = np > 1;   // else finished by the partition kernel
     float lsum = 0.f;
     float acc[PER_LANE];
 #pragma unroll
     for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
-    for (int base = 0; base < np; base += 32) {
-      const int i = base + lane;
-      const float w = i < np ? ex2(m[i] - M) : 0.f;
-      lsum += i < np ? w * l[i] : 0.f;
-      const int n = min(32, np - base);
-      int k = 0;
-      for (; k + 4 <= n; k += 4) {   // four partials in flight
-        float x[4][PER_LANE];
+    if (split) {
+      const float *m = p.ws_m + row * p.max_partitions;
+      const float *l = p.ws_l + row * p.max_partitions;
+      const float *o = p.ws_o + row * p.max_partitions * D + lane * PER_LANE;
+      float M = -INFINITY;
+      for (int i = lane; i < np; i += 32) M = fmaxf(M, m[i]);
+      M = warp_max(M);
+      for (int i0 = sub; i0 < np; i0 += kReduceBatch * wpr) {
+        // the batch's m and l: lane u < kReduceBatch loads those of partition
+        // i0 + u * wpr, then they are broadcast -- no thread reads two adjacent
+        // partials, so no load of them can be merged into a wider one (a row's
+        // m and l start only 4 * NP-byte aligned)
+        const int iu = i0 + (lane % kReduceBatch) * wpr;
+        const float m_u = lane < kReduceBatch && iu < np ? m[iu] : -INFINITY;
+        const float l_u = lane < kReduceBatch && iu < np ? l[iu] : 0.f;
+        float w[kReduceBatch], li[kReduceBatch], x[kReduceBatch][PER_LANE];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float *src = o + static_cast<size_t>(base + k + u) * D;
+        for (int u = 0; u < kReduceBatch; ++u) {   // every load of the batch in flight
+          const int i = i0 + u * wpr;
+          w[u] = __shfl_sync(kFullMask, m_u, u);
+          li[u] = __shfl_sync(kFullMask, l_u, u);
+          const float *src = o + static_cast<size_t>(i < np ? i : 0) * D;
           if constexpr (PER_LANE == 4) {
             const float4 v = *reinterpret_cast<const float4 *>(src);
             x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
@@ -981,27 +999,36 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(con
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float wk = __shfl_sync(kFullMask, w, k + u);
+        for (int u = 0; u < kReduceBatch; ++u) {
+          const float wk = ex2(w[u] - M);   // 0 past the end (m = -inf)
+          lsum += wk * li[u];
 #pragma unroll
           for (int e = 0; e < PER_LANE; ++e) acc[e] += wk * x[u][e];
         }
       }
-      for (; k < n; ++k) {
-        const float wk = __shfl_sync(kFullMask, w, k);
-        const float *src = o + static_cast<size_t>(base + k) * D;
-#pragma unroll
-        for (int e = 0; e < PER_LANE; ++e) acc[e] += wk * src[e];
-      }
     }
+    if (wpr > 1) {   // join the row's warps
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, off);
-    const float inv = 1.f / lsum;
-    T *out = reinterpret_cast<T *>(p.out) + row * D + lane * PER_LANE;
-    if constexpr (PER_LANE == 4) {
-      Elem<T>::store4(out, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    } else {
-      Elem<T>::store2(out, acc[0] * inv, acc[1] * inv);
+      for (int e = 0; e < PER_LANE; ++e) acc_s[warp][lane * PER_LANE + e] = acc[e];
+      if (lane == 0) l_s[warp] = lsum;
+      __syncthreads();
+      if (sub == 0 && split) {
+        for (int k = 1; k < wpr; ++k) {
+          lsum += l_s[warp + k];
+#pragma unroll
+          for (int e = 0; e < PER_LANE; ++e) acc[e] += acc_s[warp + k][lane * PER_LANE + e];
+        }
+      }
+      __syncthreads();   // acc_s is rewritten by the next rows
+    }
+    if (sub == 0 && split) {
+      const float inv = 1.f / lsum;
+      T *out = reinterpret_cast<T *>(p.out) + row * D + lane * PER_LANE;
+      if constexpr (PER_LANE == 4) {
+        Elem<T>::store4(out, acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      } else {
+        Elem<T>::store2(out, acc[0] * inv, acc[1] * inv);
+      }
     }
   }
 }

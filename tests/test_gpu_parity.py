@@ -119,6 +119,21 @@ def test_split_k_partition_sizes(pa, orc, P):
     assert_decode_close(out, ref, "bf16", f"P={P}")
 
 
+@pytest.mark.parametrize("np_max", [2, 3, 5, 9, 17, 33, 65])
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("bf16", 128)])
+def test_split_k_reduce_paths(pa, orc, np_max, dtype, D):
+    """Every way the reduce splits a row's partitions over warps (1, 2, 4 or 8
+    warps a row, chosen from the longest context's partition count), with rows
+    of 1 .. np_max partitions side by side; odd partition counts leave each
+    row's partials at every alignment."""
+    P = 64
+    lens = [P * np_max, P * np_max - 5, P + 1, P, 1, P * (np_max // 2) + 3, 2 * P + 7, max(1, P * np_max - 63)]
+    cfg = inputs.DecodeConfig(f"reduce_{dtype}", 9, len(lens), 8, 2, D, dtype)
+    case = inputs.make_case(cfg, lens=lens)
+    out, _ = gpu_step(pa, case, partition_size=P)
+    assert_decode_close(out, orc.decode_case(case), dtype, f"{np_max} partitions, {dtype}")
+
+
 @pytest.mark.parametrize("dtype,D", [("f32", 64), ("f16", 128), ("bf16", 128)])
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 def test_group_sizes_and_dtypes(pa, orc, dtype, D, group):
