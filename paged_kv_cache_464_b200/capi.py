@@ -210,8 +210,10 @@ def decode_static_workspace(q: torch.Tensor, k_cache: torch.Tensor, v_cache: tor
     scratch is the library's own fixed array (STATIC_WORKSPACE_BYTES per GPU),
     so the library allocates nothing.  ``out`` must be given by such callers
     (it is allocated here only as a convenience when omitted).  Calls that
-    overlap on the GPU share the array and race; the first call on a device
-    looks up the array's address and should precede any stream capture."""
+    overlap on the GPU share the array and race.  Every call that needs scratch
+    looks up the array's address on the current device (the first lookup may
+    load the library's device code there, so make the first call on each
+    device before any stream capture)."""
     nb, bs, hkv, d, dt = _cache_args(k_cache, v_cache)
     S, hq, dq = q.shape
     if dq != d or q.dtype != k_cache.dtype:
