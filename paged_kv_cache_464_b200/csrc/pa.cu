@@ -180,11 +180,11 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, 
   return w;
 }
 
-template <typename T, int G, typename Math>
+template <typename T, int G, typename Math, int W = pa::kDecodeWarps>
 pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
                           cudaStream_t stream) {
-  using SM = pa::DecodeSmem<T, G, Math>;
-  auto kernel = pa::pa_decode_partition_kernel<T, G, Math>;
+  using SM = pa::DecodeSmem<T, G, Math, W>;
+  auto kernel = pa::pa_decode_partition_kernel<T, G, Math, W>;
   // the attribute is per device; setting it on every call costs ~a microsecond of host time
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
     return PA_ERR_CUDA;
@@ -197,7 +197,7 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
     pa_status_t st = launch(pa::zero_counts_kernel, dim3((unsigned)ctas), dim3(256), 0, stream, p.ws_count, n);
     if (st != PA_OK) return st;
   }
-  pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(pa::kDecodeThreads), SM::kAlloc, stream, mk, mv, p);
+  pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(W * 32), SM::kAlloc, stream, mk, mv, p);
   if (st != PA_OK || p.max_partitions <= 1 || p.ws_count != nullptr) return st;
   // warps per row: one per 8 partitions (at most kReduceWarps); a CTA takes
   // kReduceWarps / wpr rows at a time, the grid strides over the rest (at most
@@ -212,6 +212,17 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
                 wpr);
 }
 
+// The tensor-core block math of a call that splits its sequences into
+// partitions of at most 512 tokens runs as two-warp CTAs, six an SM (short
+// CTAs: more of them resident hide more of each one's prologue and
+// epilogue); every other call as four-warp CTAs, three an SM (see
+// pa_decode.cuh).
+template <typename T, int G, typename Math>
+pa_status_t launch_mma(const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p, cudaStream_t s) {
+  if (p.max_partitions > 1 && p.partition_size <= 512) return launch_decode<T, G, Math, 2>(mk, mv, p, s);
+  return launch_decode<T, G, Math>(mk, mv, p, s);
+}
+
 // fp32 caches and single-head groups run on the CUDA cores; 16-bit caches with
 // grouped heads run the tensor-core block math.
 template <typename T>
@@ -221,13 +232,13 @@ pa_status_t dispatch_group(int group, const CUtensorMap &mk, const CUtensorMap &
   switch (group) {
     case 1: return launch_decode<T, 1, pa::FmaMath<T, 1>>(mk, mv, p, s);
     case 2:
-      if constexpr (kMma) return launch_decode<T, 2, pa::MmaMath<T, 2>>(mk, mv, p, s);
+      if constexpr (kMma) return launch_mma<T, 2, pa::MmaMath<T, 2>>(mk, mv, p, s);
       else return launch_decode<T, 2, pa::FmaMath<T, 2>>(mk, mv, p, s);
     case 4:
-      if constexpr (kMma) return launch_decode<T, 4, pa::MmaMath<T, 4>>(mk, mv, p, s);
+      if constexpr (kMma) return launch_mma<T, 4, pa::MmaMath<T, 4>>(mk, mv, p, s);
       else return launch_decode<T, 4, pa::FmaMath<T, 4>>(mk, mv, p, s);
     case 8:
-      if constexpr (kMma) return launch_decode<T, 8, pa::MmaMath<T, 8>>(mk, mv, p, s);
+      if constexpr (kMma) return launch_mma<T, 8, pa::MmaMath<T, 8>>(mk, mv, p, s);
       else return launch_decode<T, 8, pa::FmaMath<T, 8>>(mk, mv, p, s);
   }
   return PA_ERR_SHAPE;

@@ -16,7 +16,12 @@
 //   (running max m, sum l, vector o) in the workspace and the reduce kernel
 //   combines them.  A sequence that fits in one partition is finished here.
 //
-// Inside a CTA (kDecodeWarps warps, no producer warp)
+// Inside a CTA (W warps, no producer warp; W = kDecodeWarps = 4, or 2 for the
+// tensor-core block math when a call splits its sequences into partitions of
+// at most 512 tokens: then six two-warp CTAs share an SM instead of three
+// four-warp ones, which hides more of each CTA's fixed cost -- measured on B200
+// 169.6 against 172.9 µs a call on the long-context workload, while the GQA
+// workload with 1024-token partitions is 2% faster with four warps)
 //   Warp w owns the partition's blocks w, w+W, w+2W, ... and keeps its own
 //   online-softmax state.  Each warp has kStagesPerWarp shared-memory stages;
 //   one elected lane issues a TMA tensor load for the K tile and the V tile of
@@ -628,20 +633,20 @@ struct Fp8MmaMath {
 };
 
 // ============================================================ shared memory plan
-template <typename T, int G, typename Math>
+template <typename T, int G, typename Math, int W = kDecodeWarps>
 struct DecodeSmem {
   static constexpr int D = Math::D;
   static constexpr int kTile = kBlockSize * Math::kRowBytes;        // one K or V tile
-  static constexpr int kStages = kDecodeWarps * Math::kStagesPerWarp;
+  static constexpr int kStages = W * Math::kStagesPerWarp;
   static constexpr int kTilesBytes = kStages * 2 * kTile;
   static constexpr int kScratchOff = kTilesBytes;
   static constexpr int kMOff = kScratchOff + Math::kScratchBytes;
-  static constexpr int kLOff = kMOff + kDecodeWarps * G * 4;
-  static constexpr int kFlagOff = kLOff + kDecodeWarps * G * 4;
+  static constexpr int kLOff = kMOff + W * G * 4;
+  static constexpr int kFlagOff = kLOff + W * G * 4;
   static constexpr int kBarOff = (kFlagOff + 8 + 7) / 8 * 8;   // abort flag, last-partition flag
   static constexpr int kBytes = kBarOff + kStages * 8;
   static constexpr int kAlloc = kBytes + 1024;   // room to align the base to 1024 B (128B swizzle atom)
-  static_assert(kDecodeWarps * G * D * 4 <= kTilesBytes, "epilogue buffer must fit in the stage tiles");
+  static_assert(W * G * D * 4 <= kTilesBytes, "epilogue buffer must fit in the stage tiles");
 };
 
 // ============================================================ split-K combine
@@ -653,11 +658,11 @@ struct DecodeSmem {
 // lane-strided max and sum over the partitions joined by shuffles, then o
 // accumulated over the partitions in order.  Partials are read through L2
 // (.cg): other SMs wrote them.
-template <typename T, int G, int D>
+template <typename T, int G, int D, int W>
 __device__ __forceinline__ void combine_partitions(const DecodeParams &p, int b, int h0, int nparts, float *M_s,
                                                    float *inv_s, T *out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int hh = warp; hh < G; hh += kDecodeWarps) {
+  for (int hh = warp; hh < G; hh += W) {
     const size_t row = static_cast<size_t>(b) * p.num_heads + h0 + hh;
     const float *m = p.ws_m + row * p.max_partitions;
     const float *l = p.ws_l + row * p.max_partitions;
@@ -674,7 +679,7 @@ __device__ __forceinline__ void combine_partitions(const DecodeParams &p, int b,
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x * 4; i < G * D; i += kDecodeThreads * 4) {
+  for (int i = threadIdx.x * 4; i < G * D; i += W * 32 * 4) {
     const int hh = i / D, d = i % D;
     const size_t row = static_cast<size_t>(b) * p.num_heads + h0 + hh;
     const float *m = p.ws_m + row * p.max_partitions;
@@ -721,11 +726,16 @@ __global__ void __launch_bounds__(256) zero_counts_kernel(unsigned *count, int n
 }
 
 // ============================================================ partition kernel
-template <typename T, int G, typename Math>
-__global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
+// Resident CTAs an SM the register budget is sized for: four-warp CTAs (the
+// default launch shape), or six of the two-warp shape.
+constexpr int decode_min_ctas(int warps) { return warps == 2 ? 6 : PA_DECODE_MIN_CTAS_PER_SM; }
+
+template <typename T, int G, typename Math, int W = kDecodeWarps>
+__global__ void __launch_bounds__(W * 32, decode_min_ctas(W))
     pa_decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                const DecodeParams p) {
-  using SM = DecodeSmem<T, G, Math>;
+  static_assert(!Math::kNeedsQInSmem || W == kDecodeWarps, "the CUDA-core block math stages q with kDecodeWarps warps");
+  using SM = DecodeSmem<T, G, Math, W>;
   constexpr int D = SM::D;
   constexpr int kTile = SM::kTile;
   constexpr int kStages = SM::kStages;
@@ -764,7 +774,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   T *out = reinterpret_cast<T *>(p.out) + (static_cast<size_t>(b) * p.num_heads + h0) * D;
   if (L == 0) {   // empty context: the row is the empty sum, zeros
     if (part == 0)
-      for (int i = threadIdx.x * 4; i < G * D; i += kDecodeThreads * 4) Elem<T>::store4(out + i, 0.f, 0.f, 0.f, 0.f);
+      for (int i = threadIdx.x * 4; i < G * D; i += (W * 32) * 4) Elem<T>::store4(out + i, 0.f, 0.f, 0.f, 0.f);
     return;
   }
   if (part >= nparts) return;
@@ -782,7 +792,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   }
 
   // ---- this warp's blocks: local block index warp + j * W, j = 0 .. nw-1
-  const int nw = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+  const int nw = nblk > warp ? (nblk - warp + W - 1) / W : 0;
   const int32_t *bt_row = p.block_tables + static_cast<size_t>(b) * p.max_blocks_per_seq + tok0 / kBlockSize;
   int id_group = -1;   // which 32 consecutive j's the lanes' ids belong to
   int my_id = -1;      // lane l holds the physical id of j = 32 * id_group + l
@@ -794,13 +804,13 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
       const int jj = (id_group << 5) + lane;
       my_id = -1;
       if (jj < nw) {
-        const int id = bt_row[warp + jj * kDecodeWarps];
+        const int id = bt_row[warp + jj * W];
         if (id < 0 || id >= p.num_blocks) record_error(1 /*PA_DEV_BAD_BLOCK_ID*/, id);
         else my_id = id;
       }
     }
     const int id = __shfl_sync(kFullMask, my_id, j & 31);
-    const int s = warp + (j % kSPW) * kDecodeWarps;
+    const int s = warp + (j % kSPW) * W;
     if (lane == 0 && !(stall_here && warp == 0 && j == 0)) {   // (test hook: warp 0's first stage left unissued)
       if (id >= 0) {
         // one box per 128-byte part of the rows: the tile lands as [part][token][128 B]
@@ -828,7 +838,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   bool ok = true;
   int j = 0;
   for (; j < nw; ++j) {
-    const int s = warp + (j % kSPW) * kDecodeWarps;
+    const int s = warp + (j % kSPW) * W;
     const bool landed = mbar_wait(&full[s], (j / kSPW) & 1, wait_limit);
     if (!__all_sync(kFullMask, landed)) {
       if (lane == 0) {
@@ -839,7 +849,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
       break;
     }
     uint8_t *tk = smem + s * 2 * kTile;
-    const int lb = warp + j * kDecodeWarps;   // local block index
+    const int lb = warp + j * W;   // local block index
     const int nvalid = min(kBlockSize, tok1 - (tok0 + lb * kBlockSize));
     if (Math::kRowBytes == 256 && p.new_k != nullptr && part == nparts - 1 && lb == nblk - 1) {
       // append mode: this block holds position L-1.  Store the new token's K/V
@@ -873,7 +883,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
     // the stages of blocks j .. j + kSPW - 1, the one that timed out included
     // (its copy may still arrive)
     for (int jj = j; jj < min(nw, j + kSPW); ++jj)
-      mbar_wait(&full[warp + (jj % kSPW) * kDecodeWarps], (jj / kSPW) & 1, wait_limit);
+      mbar_wait(&full[warp + (jj % kSPW) * W], (jj / kSPW) & 1, wait_limit);
   }
 
   // ---- merge the warps through shared memory (the stage tiles are reused)
@@ -883,15 +893,15 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   __syncthreads();
   if (*abort_s) return;
 
-  for (int i = threadIdx.x * 4; i < G * D; i += kDecodeThreads * 4) {
+  for (int i = threadIdx.x * 4; i < G * D; i += (W * 32) * 4) {
     const int hh = i / D, d = i % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, m_s[w * G + hh]);
+    for (int w = 0; w < W; ++w) M = fmaxf(M, m_s[w * G + hh]);
     float lsum = 0.f;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) {
+    for (int w = 0; w < W; ++w) {
       const float f = ex2(m_s[w * G + hh] - M);   // 0 for a warp that saw no token
       lsum += f * l_s[w * G + hh];
       const float4 x = *reinterpret_cast<const float4 *>(o_s + (w * G + hh) * D + d);
@@ -924,7 +934,7 @@ __global__ void __launch_bounds__(kDecodeThreads, PA_DECODE_MIN_CTAS_PER_SM)
   __syncthreads();
   if (!*last_s) return;
   __threadfence();   // the other CTAs' partials (published before their tickets) are visible from here on
-  combine_partitions<T, G, D>(p, b, h0, nparts, m_s, l_s, out);
+  combine_partitions<T, G, D, W>(p, b, h0, nparts, m_s, l_s, out);
 }
 
 // Combine the partitions of every (sequence, query head) that was split:
