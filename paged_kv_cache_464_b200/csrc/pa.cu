@@ -17,6 +17,7 @@
 #include "pa_cache_ops.cuh"
 #include "pa_decode.cuh"
 #include "pa_prefill.cuh"
+#include "pa_decode_fp8tc.cuh"
 #include "pa_probe.cuh"
 
 #ifndef PA_PROGRAMMATIC_LAUNCH
@@ -180,6 +181,9 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, 
   return w;
 }
 
+template <typename T>
+pa_status_t launch_reduce(const pa::DecodeParams &p, cudaStream_t stream);
+
 template <typename T, int G, typename Math, int W = pa::kDecodeWarps>
 pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
                           cudaStream_t stream) {
@@ -199,6 +203,12 @@ pa_status_t launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pa
   }
   pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(W * 32), SM::kAlloc, stream, mk, mv, p);
   if (st != PA_OK || p.max_partitions <= 1 || p.ws_count != nullptr) return st;
+  return launch_reduce<T>(p, stream);
+}
+
+// Split-K reduce of a decode call's partials (after its partition kernel).
+template <typename T>
+pa_status_t launch_reduce(const pa::DecodeParams &p, cudaStream_t stream) {
   // warps per row: one per 8 partitions (at most kReduceWarps); a CTA takes
   // kReduceWarps / wpr rows at a time, the grid strides over the rest (at most
   // 8 CTAs of 8 warps per SM)
@@ -244,10 +254,45 @@ pa_status_t dispatch_group(int group, const CUtensorMap &mk, const CUtensorMap &
   return PA_ERR_SHAPE;
 }
 
-// 1-byte E4M3 caches: tensor-core block math in fp16 for every group size
+// E4M3 caches on the tcgen05 path (pa_decode_fp8tc.cuh): the same grid and
+// partials as launch_decode, combined by the same reduce.
+template <typename T, int G>
+pa_status_t launch_fp8tc(const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p0,
+                         cudaStream_t stream) {
+  using SH = pa::Fp8TcShape<G>;
+  auto kernel = pa::pa_decode_fp8tc_kernel<T, G>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::kAlloc) != cudaSuccess)
+    return PA_ERR_CUDA;
+  pa::DecodeParams p = p0;
+  p.ws_count = nullptr;   // partials always combined by the reduce kernel
+  const long long grid = (long long)p.num_seqs * p.num_kv_heads * p.max_partitions;
+  if (grid == 0) return PA_OK;
+  if (grid > INT32_MAX) return PA_ERR_SHAPE;
+  pa_status_t st = launch(kernel, dim3((unsigned)grid), dim3(pa::kTcThreads), SH::kAlloc, stream, mk, mv, p);
+  if (st != PA_OK || p.max_partitions <= 1) return st;
+  return launch_reduce<T>(p, stream);
+}
+
+// 1-byte E4M3 caches: the mma.sync block math in fp16 with the codes
+// converted on the CUDA cores (the default), or, built with PA_FP8_TC=1, the
+// tcgen05 kernel whose tensor cores read the codes as they land (parity-green,
+// measured 1.45x slower on B200: each 128-token tile waits on a serial chain of
+// products, softmax and hand-overs, so too few tiles are in flight an SM)
+#ifndef PA_FP8_TC
+#define PA_FP8_TC 0
+#endif
 template <typename T>
 pa_status_t dispatch_group_fp8(int group, const CUtensorMap &mk, const CUtensorMap &mv, const pa::DecodeParams &p,
                                cudaStream_t s) {
+  if (PA_FP8_TC) {
+    switch (group) {
+      case 1: return launch_fp8tc<T, 1>(mk, mv, p, s);
+      case 2: return launch_fp8tc<T, 2>(mk, mv, p, s);
+      case 4: return launch_fp8tc<T, 4>(mk, mv, p, s);
+      case 8: return launch_fp8tc<T, 8>(mk, mv, p, s);
+    }
+    return PA_ERR_SHAPE;
+  }
   switch (group) {
     case 1: return launch_decode<T, 1, pa::Fp8MmaMath<T, 1>>(mk, mv, p, s);
     case 2: return launch_decode<T, 2, pa::Fp8MmaMath<T, 2>>(mk, mv, p, s);

@@ -82,6 +82,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   }
 }
 
+// Non-blocking: has phase `parity` of `bar` completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait (`limit_ns`) that also gives up once another role has raised
+// the abort flag.  With `backoff` the waiting warp sleeps between polls,
+// leaving the shared memory ports (which also feed the tensor cores' operands)
+// to others.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, const volatile int *abort_flag,
+                                                   unsigned long long limit_ns, bool backoff = false) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (backoff) __nanosleep(64);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && (*abort_flag || global_ns() - t0 > limit_ns)) return false;
+  }
+}
+
 // Test hook for the bounded-wait error path.  A kernel launched with
 // stall_cta = c + 1 (0 = off, the value of every ordinary launch) treats its CTA
 // c specially: that CTA leaves one of its copies unissued -- no copy and no

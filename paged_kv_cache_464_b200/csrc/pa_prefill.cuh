@@ -157,32 +157,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Non-blocking: has phase `parity` of `bar` completed?
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-// Bounded wait (`limit_ns`) that also gives up once another role has raised
-// the abort flag.  With `backoff` the waiting warp sleeps between polls,
-// leaving the shared memory ports (which also feed the tensor cores' operands)
-// to others.
-__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, const volatile int *abort_flag,
-                                                   unsigned long long limit_ns, bool backoff = false) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (backoff) __nanosleep(64);
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && (*abort_flag || global_ns() - t0 > limit_ns)) return false;
-  }
-}
-
 template <typename T, int G>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     pa_prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,

@@ -6,7 +6,8 @@
 // offset >> 4 at bit 16, stride byte offset >> 4 at bit 32, version 1 at bit
 // 46, layout type at bit 61; instruction descriptor for kind::f16: accumulator
 // format at bit 4, A / B formats at bits 7 / 10, A / B major at bits 15 / 16,
-// N >> 3 at bit 17, M >> 4 at bit 24).  Included only from pa.cu.
+// N >> 3 at bit 17, M >> 4 at bit 24; kind::f8f6f4 has the same fields, E4M3
+// being format 0).  Included only from pa.cu.
 #pragma once
 
 #include "pa_common.cuh"
@@ -35,6 +36,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void *start, uint32_t 
 __host__ __device__ constexpr uint32_t instr_desc_f16(int ab_format, bool b_mn_major, int M, int N) {
   return (1u << 4) | ((uint32_t)ab_format << 7) | ((uint32_t)ab_format << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// kind::f8f6f4 instruction descriptor with both operands E4M3 (format 0) and an
+// fp32 accumulator; A and B each K-major or MN-major.
+__host__ __device__ constexpr uint32_t instr_desc_e4m3(bool a_mn_major, bool b_mn_major, int M, int N) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 
 // ---------------------------------------------------------------- tensor memory
@@ -77,6 +85,17 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// D (tensor memory) (+)= A (smem) * B (smem), 8-bit operands (K = 32 a product);
+// issued by one thread.
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1 : 0)
+      : "memory");
+}
+
 // Arrive once on `bar` when all earlier tcgen05 operations of this thread complete.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
@@ -98,6 +117,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // 32 consecutive 32-bit columns of this thread's lane from raw words.

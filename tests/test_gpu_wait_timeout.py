@@ -151,3 +151,48 @@ def test_prefill_wait_runs_out_in_one_cta(pa, orc):
     code, detail = pa.get_device_error(clear=True)
     assert code == 0, (code, detail)
     _close(out2.to(torch.float64).cpu().numpy(), ref, "next launch")
+
+
+def _fp8_codes(orc, case, k_scale, v_scale):
+    """1-byte caches holding every attended token of a 16-bit case (quantised by the oracle)."""
+    NB, bs, Hkv, D = case.k_cache_post.shape
+    sm = torch.cat([case.block_tables[b, torch.arange(int(L)) // bs].to(torch.int64) * bs + torch.arange(int(L)) % bs
+                    for b, L in enumerate(case.context_lens.tolist())])
+    K = case.k_cache_post.view(NB * bs, Hkv, D)[sm].contiguous()
+    V = case.v_cache_post.view(NB * bs, Hkv, D)[sm].contiguous()
+    kc = torch.zeros((NB, bs, Hkv, D), dtype=torch.uint8)
+    vc = torch.zeros_like(kc)
+    assert orc.reshape_and_cache_fp8(kc, vc, K, V, sm, k_scale, v_scale) == 0
+    return kc, vc
+
+
+def test_fp8_decode_wait_runs_out_in_one_cta(pa, orc):
+    # the tensor-core E4M3 kernel: the stalled CTA's TMA warp leaves its first
+    # tile unissued, so the issuer's wait on it runs out and every role stops
+    case = inputs.make_case("llama3_8b_gqa", lens=[128, 700, 1000, 33])
+    cfg = case.cfg
+    G, Hkv = cfg.group, cfg.num_kv_heads
+    ks, vs = 0.0125, 0.011
+    kc, vc = _fp8_codes(orc, case, ks, vs)
+    ref = orc.paged_decode_fp8(case.q, kc, vc, ks, vs, case.block_tables, case.context_lens, case.scale)
+    dev = "cuda"
+    args = [case.q.to(dev), kc.to(dev), vc.to(dev), ks, vs, case.block_tables.to(dev), case.context_lens.to(dev),
+            case.scale]
+    b, g = 2, 6
+    cta = b * Hkv + g                # one partition a sequence (P = 1024)
+    out = torch.full_like(args[0], SENTINEL)
+    pa.get_device_error(clear=True)
+    pa.test_stall_next_launch("decode", cta)
+    pa.decode_fp8(*args, out, max_context_len=case.max_context_len)
+    code, detail = pa.get_device_error(clear=True)
+    assert (code, detail) == (PA_DEV_WAIT_TIMEOUT, cta)
+    got = out.to(torch.float64).cpu().numpy()
+    heads = slice(g * G, (g + 1) * G)
+    assert (got[b, heads] == SENTINEL).all(), "the stalled CTA wrote its rows"
+    mask = np.ones(got.shape[:2], dtype=bool)
+    mask[b, heads] = False
+    _close(got[mask], ref[mask], "other rows of the stalled launch")
+    out2 = pa.decode_fp8(*args, max_context_len=case.max_context_len)
+    code, detail = pa.get_device_error(clear=True)
+    assert code == 0, (code, detail)
+    _close(out2.to(torch.float64).cpu().numpy(), ref, "next launch")
