@@ -78,6 +78,8 @@ typedef enum {
   PA_DEV_BAD_CONTEXT_LEN = 4,  /* context_len < 0, > max_context_len or > table capacity; detail = seq */
   PA_DEV_WAIT_TIMEOUT = 5,     /* an internal bounded wait gave up; detail = linear CTA index
                                   (blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) */
+  PA_DEV_VALUE_RANGE = 6,      /* pa_prefill, bf16 caches: an attended V element with |v| >= 2^24
+                                  (outside the kernel's fp16 range for V); detail = sequence */
 } pa_device_error_t;
 
 /*
@@ -237,10 +239,14 @@ pa_status_t pa_decode_append(void *out, const void *q, const void *key, const vo
  * max_query_len     an upper bound of every n_b (sizes the grid).
  * Other arguments as pa_decode.  head_dim must be 128 and G one of 1, 2, 4, 8.
  * Computed on the tensor cores (tcgen05) with fp32 accumulation; the softmax
- * weights enter P V as two 16-bit parts (hi + lo), so accuracy is that of
- * pa_decode.  Device-side errors: PA_DEV_BAD_CONTEXT_LEN (n_b < 0, n_b >
- * max_query_len, L_b < n_b or L_b > max_blocks_per_seq * 16: sequence skipped),
- * PA_DEV_BAD_BLOCK_ID (the block reads as zeros), PA_DEV_WAIT_TIMEOUT.
+ * weights enter P V as fp16 (relative rounding <= 2^-11), and so does V: bf16
+ * caches are converted in shared memory, scaled by 2^-8 (exact for every bf16
+ * |v| < 2^24; smaller magnitudes keep an absolute accuracy of 2^-17), the
+ * scale undone in the output.  Device-side errors: PA_DEV_BAD_CONTEXT_LEN (n_b
+ * < 0, n_b > max_query_len, L_b < n_b or L_b > max_blocks_per_seq * 16:
+ * sequence skipped), PA_DEV_BAD_BLOCK_ID (the block reads as zeros),
+ * PA_DEV_VALUE_RANGE (bf16 only: a V element at or above 2^24 in magnitude;
+ * that sequence's outputs are not valid), PA_DEV_WAIT_TIMEOUT.
  * Errors: PA_ERR_NULL, PA_ERR_DTYPE, PA_ERR_SHAPE, PA_ERR_ALIGN, PA_ERR_CUDA.
  * num_seqs == 0 or max_query_len == 0 is a no-op.
  */

@@ -18,24 +18,30 @@
 // (row = query * G + head), so every K/V tile read from the cache serves all
 // grouped heads, and the two query tiles of a CTA share every K/V tile.  The
 // KV walk runs over tiles of 64 tokens (four cache blocks) up to the last
-// query's position.  Warp roles (384 threads):
+// query's position.  Warp roles (512 threads):
 //   warps 0-3, 4-7  one softmax warpgroup per query tile; thread = row.  Per KV
 //                   tile: tcgen05.ld of its 64 scores, causal mask on diagonal
 //                   tiles, online max/sum in base 2 (O rescaled in tensor
 //                   memory only when a row's max grows by more than 2^8), P
-//                   written back over its scores in tensor memory as two
-//                   16-bit parts hi + lo (P carries ~15 bits or more, like the
-//                   decode kernel);
+//                   written back over its scores in tensor memory as fp16
+//                   (relative rounding <= 2^-11);
 //   warps 8, 10     tensor-core issue, one thread per query tile: S = Q K^T
 //                   (M=128 N=64, 8 x K=16, both operands in shared memory)
-//                   into a double-buffered S, and O += P_hi V + P_lo V (M=128
-//                   N=128, 2 x 4 x K=16, P read from tensor memory, V from
-//                   shared memory), QK(j+1) before PV(j); the tensor pipe runs
-//                   one query tile's products while the other's issuer waits;
+//                   into a double-buffered S, and O += P V (M=128 N=128,
+//                   4 x K=16, fp16, P read from tensor memory, V from shared
+//                   memory), QK(j+1) before PV(j); the tensor pipe runs one
+//                   query tile's products while the other's issuer waits.  A
+//                   product costs about the same below N=256 whatever its
+//                   width, so the kernel is bound by its count of products:
+//                   one fp16 pass of P V instead of two bf16 ones (hi + lo)
+//                   takes a quarter of them away;
 //   warp 9          TMA: K and V tiles (four 2 KiB boxes per 128-byte half of
 //                   the rows, 128-byte swizzled) into rings of 3 stages each,
 //                   block ids read from the block table one per lane;
-//   warp 11         idle (as are lanes 1-31 of warps 8 and 10).
+//   warps 12-15     bf16 caches: rewrite each landed V tile in place as fp16
+//                   times 2^-8 (exact for |v| < 2^24) and zero the rows past
+//                   the context end, then hand it to the issuers; f16 caches:
+//                   idle (as are warp 11 and lanes 1-31 of warps 8 and 10).
 // Roles hand over through mbarriers (one arrival per warp) only; every wait is
 // bounded, and a role that gives up raises a CTA-wide abort so that the others
 // stop waiting.  Each barrier is waited on by parity, so no barrier may complete
@@ -45,7 +51,7 @@
 // PV(j) has seen S(j+1), which needed PV(j-2) done); the K/V ring barriers
 // advance one phase per hand-over that their waiter itself enables.
 // Tensor memory: per query tile, S[2] (2 x 64 columns; P of a tile replaces
-// its S: 32 columns of hi pairs, then 32 of lo pairs) and O (128 columns).
+// the first 32 columns of its S as fp16 pairs) and O (128 columns).
 #pragma once
 
 #include "pa_common.cuh"
@@ -69,9 +75,11 @@ constexpr int kPrefillRows = 128;        // M: rows of one query tile
 constexpr int kPrefillTiles = 2;         // query tiles (softmax warpgroups) per CTA
 constexpr int kPrefillMmaWarp = 4 * kPrefillTiles;
 constexpr int kPrefillLoadWarp = kPrefillMmaWarp + 1;
-// three whole warpgroups: warps 10-11 only join the CTA barriers (ptxas fits
-// the softmax in the 168 registers of a 384-thread block without spilling)
-constexpr int kPrefillThreads = 128 * (kPrefillTiles + 1);
+constexpr int kPrefillConvWarp = 4 * (kPrefillTiles + 1);   // first of the four V converter warps
+constexpr int kPrefillConvWarps = 4;
+// four whole warpgroups: two softmax, one for the issuers and the TMA warp
+// (warp 11 idle), one converting bf16 V tiles (idle for f16 caches)
+constexpr int kPrefillThreads = 128 * (kPrefillTiles + 2);
 constexpr int kPrefillKv = 64;           // N of S = Q K^T: tokens per KV tile
 constexpr int kPrefillKStages = 3;
 constexpr int kPrefillVStages = 3;
@@ -86,9 +94,10 @@ struct PrefillSmem {
   static constexpr int kK = kQ + kPrefillTiles * kQTileBytes;
   static constexpr int kV = kK + kPrefillKStages * kKvTileBytes;
   static constexpr int kBar = kV + kPrefillVStages * kKvTileBytes;
-  // k_full[KS] v_full[VS] k_free[KS] v_free[VS]; per query tile: s_full[2] p_full[2] o_done[2]; drain, tail_ready
+  // k_full[KS] v_full[VS] k_free[KS] v_free[VS]; per query tile: s_full[2] p_full[2] o_done[2]; drain,
+  // tail_ready; v_conv[VS]
   static constexpr int kTileBars = 6;
-  static constexpr int kNumBars = 2 * (kPrefillKStages + kPrefillVStages) + kPrefillTiles * kTileBars + 2;
+  static constexpr int kNumBars = 2 * (kPrefillKStages + kPrefillVStages) + kPrefillTiles * kTileBars + 2 + kPrefillVStages;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
   static constexpr int kFlag = kTmemSlot + 4;
   static constexpr int kBytes = kFlag + 4;
@@ -100,18 +109,8 @@ template <typename T>
 struct Pack16;
 template <>
 struct Pack16<__nv_bfloat16> {
-  static constexpr int kFormat = 1;   // tcgen05 kind::f16 operand format
-  // p = hi + lo + t: hi = the top 16 bits of p (p truncated to bf16), lo = the
-  // top 16 bits of the exact remainder p - hi; |t| < 2^-15 |p|.  Integer
-  // work only (no conversion instructions); two values per 32-bit word, the
-  // first in the low half.
-  __device__ __forceinline__ static void split(float2 e, uint32_t &hi, uint32_t &lo) {
-    const uint32_t ua = __float_as_uint(e.x), ub = __float_as_uint(e.y);
-    hi = __byte_perm(ua, ub, 0x7632);
-    const float2 r = __ffma2_rn(make_float2(__uint_as_float(ua & 0xffff0000u), __uint_as_float(ub & 0xffff0000u)),
-                                make_float2(-1.f, -1.f), e);   // e - hi, exact
-    lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
-  }
+  static constexpr int kFormat = 1;       // tcgen05 kind::f16 operand format of q and K
+  static constexpr bool kConvertV = true; // V tiles rewritten as fp16 (times 2^-8) before PV
   __device__ __forceinline__ static uint32_t pack(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -120,18 +119,19 @@ struct Pack16<__nv_bfloat16> {
 template <>
 struct Pack16<__half> {
   static constexpr int kFormat = 0;
-  __device__ __forceinline__ static void split(float2 e, uint32_t &hi, uint32_t &lo) {
-    const __half2 h = __floats2half2_rn(e.x, e.y);
-    const float2 hf = __half22float2(h);
-    const __half2 l = __floats2half2_rn(e.x - hf.x, e.y - hf.y);
-    hi = *reinterpret_cast<const uint32_t *>(&h);
-    lo = *reinterpret_cast<const uint32_t *>(&l);
-  }
+  static constexpr bool kConvertV = false; // V is fp16 already
   __device__ __forceinline__ static uint32_t pack(float a, float b) {
     __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&v);
   }
 };
+
+// Two softmax weights -> one fp16 pair (the A operand of P V), the first in the
+// low half; relative rounding <= 2^-11.
+__device__ __forceinline__ uint32_t pack_p(float2 e) {
+  __half2 v = __floats2half2_rn(e.x, e.y);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
 
 // 64 consecutive fp32 columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t *tile_bars = v_free + VS;   // query tile w: s_full[2], p_full[2], o_done[2] at w * kTileBars
   uint64_t *drain = tile_bars + NT * SM::kTileBars;
   uint64_t *tail_ready = drain + 1;
+  uint64_t *v_conv = tail_ready + 1;   // [VS] bf16 caches: V tile rewritten as fp16
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM::kTmemSlot);
   volatile int *abort_s = reinterpret_cast<int *>(smem + SM::kFlag);
 
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     mbar_init(drain, NT);
     mbar_init(tail_ready, 1);
+    for (int i = 0; i < VS; ++i) mbar_init(&v_conv[i], kPrefillConvWarps);   // one arrival per converter warp
     fence_mbar_init();
     *abort_s = 0;
   }
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int ntw = nt[w];
     uint64_t *tb = tile_bars + w * SM::kTileBars;
     constexpr uint32_t kIdescQK = instr_desc_f16(PK::kFormat, false, kPrefillRows, kPrefillKv);
-    constexpr uint32_t kIdescPV = instr_desc_f16(PK::kFormat, true, kPrefillRows, D);
+    constexpr uint32_t kIdescPV = instr_desc_f16(0 /* f16: P, and V after conversion */, true, kPrefillRows, D);
     bool ok = true;
     auto wait = [&](uint64_t *bar, uint32_t parity) {
       if (!ok) return;
@@ -391,10 +393,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       umma_commit(&k_free[j % KS]);         // this issuer is done with the K stage once they complete
     };
     auto issue_pv = [&](int j) {   // O_w += P_w(j) V_j
-      wait(&v_full[j % VS], (j / VS) & 1);
+      if constexpr (PK::kConvertV) wait(&v_conv[j % VS], (j / VS) & 1);   // rewritten as fp16, tail zeroed
+      else wait(&v_full[j % VS], (j / VS) & 1);
       if (!ok) return;
       uint8_t *vt = smem + SM::kV + (j % VS) * SM::kKvTileBytes;
-      if (zero_tail && j == ntiles - 1) {
+      if (!PK::kConvertV && zero_tail && j == ntiles - 1) {
         if (w == tail_owner) {
           // rows past the context end in its last block may hold anything (NaN
           // included); make them zero so that 0 * V stays 0
@@ -415,15 +418,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       wait(&tb[2 + (j & 1)], (j >> 1) & 1);   // P_w(j) written
       if (!ok) return;
       const uint64_t b0 = v_desc + (((j % VS) * SM::kKvTileBytes) >> 4);
-      const uint32_t a0 = tmem + w * 256 + (j & 1) * kPrefillKv;   // P_w(j): hi pairs, then lo pairs
+      const uint32_t a0 = tmem + w * 256 + (j & 1) * kPrefillKv;   // P_w(j): fp16 pairs in 32 columns
       const uint32_t o_tmem = tmem + w * 256 + 128;
       const bool acc = j > 0;
 #pragma unroll
-      for (int part = 0; part < 2; ++part)
-#pragma unroll
-        for (int kk = 0; kk < kPrefillKv / 16; ++kk)   // 16 tokens = 8 columns of P per step
-          umma_f16_ts(o_tmem, a0 + part * 32 + kk * 8, b0 + ((kk * 16 * 128) >> 4), kIdescPV,
-                      acc || part > 0 || kk > 0);
+      for (int kk = 0; kk < kPrefillKv / 16; ++kk)   // 16 tokens = 8 columns of P per step
+        umma_f16_ts(o_tmem, a0 + kk * 8, b0 + ((kk * 16 * 128) >> 4), kIdescPV, acc || kk > 0);
       umma_commit(&tb[4 + (j & 1)]);   // o_done
       umma_commit(&v_free[j % VS]);    // this issuer is done with the V stage once they complete
     };
@@ -437,6 +437,55 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (!ok) break;
       if (j < ntw) issue_pv(j);
       else free_arrive(v_free, j, VS);
+    }
+  } else if (warp >= kPrefillConvWarp) {
+    if constexpr (PK::kConvertV) {
+      // ================================================================ V converter (bf16 caches)
+      // Every landed V tile is rewritten in place as fp16 times 2^-8 (exact for
+      // |v| < 2^24, the kernel's stated range; larger magnitudes are recorded as
+      // PA_DEV_VALUE_RANGE), and the rows of tokens at or past the context end
+      // (stale slots of the last block, possibly NaN) become zero, so that
+      // 0 * V stays 0.  The element positions do not move, so the tile keeps
+      // its swizzled layout.  Four warps, 8 16-byte chunks a lane per tile;
+      // each warp arrives once on the stage's conversion barrier.
+      const int ct = (warp - kPrefillConvWarp) * 32 + lane;   // converter thread 0..127
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        ok = __all_sync(kFullMask, mbar_wait_or_abort(&v_full[j % VS], (j / VS) & 1, abort_s, wait_limit, true));
+        if (!ok) {
+          if (lane == 0) {
+            record_error(5 /*PA_DEV_WAIT_TIMEOUT*/, cta);
+            *abort_s = 1;
+          }
+          break;
+        }
+        uint4 *vt = reinterpret_cast<uint4 *>(smem + SM::kV + (j % VS) * SM::kKvTileBytes);
+        const int valid_rows = L - j * kPrefillKv;   // rows at or past this are past the context end
+        float vmax = 0.f;   // max |v| converted (fmaxf skips NaN, which passes through as NaN)
+#pragma unroll
+        for (int i = 0; i < SM::kKvTileBytes / 16 / 128; ++i) {
+          const int c = ct + 128 * i;
+          const int row = (c % (SM::kHalfBytes / 16)) >> 3;   // 8 chunks a 128-byte row, [half][row][128 B]
+          uint4 x = vt[c];
+          if (row >= valid_rows) {
+            x = make_uint4(0u, 0u, 0u, 0u);
+          } else {
+            uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xffff0000u);
+              vmax = fmaxf(vmax, fmaxf(fabsf(lo), fabsf(hi)));
+              w[k] = pack_p(make_float2(lo * 0.00390625f, hi * 0.00390625f));
+            }
+          }
+          vt[c] = x;
+        }
+        const bool range_bad = vmax >= 16777216.f;   // |v| >= 2^24
+        fence_proxy_async_smem();   // generic stores read by the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&v_conv[j % VS]);
+        if (__any_sync(kFullMask, range_bad) && lane == 0) record_error(6 /*PA_DEV_VALUE_RANGE*/, b);
+      }
     }
   } else if (warp < kPrefillMmaWarp) {
     // ================================================================ softmax warpgroup w
@@ -494,20 +543,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       const float2 nmc = make_float2(-m_run * c2, -m_run * c2);
       const float2 cc2 = make_float2(c2, c2);
-      uint32_t ph[32], pl[32];
+      uint32_t ph[32];
       float2 sum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const float2 x = __ffma2_rn(make_float2(s[2 * k], s[2 * k + 1]), cc2, nmc);
         const float2 e = make_float2(ex2(x.x), ex2(x.y));
         sum[k & 1] = __fadd2_rn(sum[k & 1], e);
-        PK::split(e, ph[k], pl[k]);
+        ph[k] = pack_p(e);
       }
       l_run += (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
 
       // -- P(j) over S(j) in tensor memory (S(j) is in registers now)
       tmem_st32u(t_s + (j & 1) * kPrefillKv, ph);
-      tmem_st32u(t_s + (j & 1) * kPrefillKv + 32, pl);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       // -- a row whose max grew: O, complete up to tile j-1, rescaled before PV(j)
       if (__any_sync(kFullMask, need)) {
@@ -530,7 +578,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // -- epilogue: O / l -> out
       wait(&tb[4 + ((ntw - 1) & 1)], ((ntw - 1) >> 1) & 1);   // the last PV (and so every PV) done
       if (ok) {
-        const float inv = 1.f / l_run;
+        const float inv = (PK::kConvertV ? 256.f : 1.f) / l_run;   // V entered P V scaled by 2^-8
         T *orow = reinterpret_cast<T *>(p.out) +
                   (static_cast<size_t>(qs + q0 + i_row) * p.num_heads + g * G + r % G) * D;
         const bool row_valid = i_row < nq;

@@ -12,7 +12,11 @@ Roles, as in the kernel:
   whose query tile does not reach a KV tile still arrives once on its stages;
 * one softmax role per query tile waits for S_w(j), sometimes rescales O (then
   waits for PV_w(j-1)), and hands P_w(j) over; the epilogue waits for the
-  last PV.
+  last PV;
+* with `convert` (bf16 caches) a converter role takes every landed V tile,
+  rewrites it in place as fp16 (and zeroes the rows past the context end of
+  the last tile), and hands it to the issuers on its own barrier per stage;
+  the issuers' PV then waits on that barrier instead of the TMA's.
 The tensor pipe starts products in issue order but overlaps them: a product
 may start before the previous one has completed (and so before it has read
 all of its operands), which is why a product that overwrites another's
@@ -47,7 +51,7 @@ class Bar:
 
 
 def run(nt_a: int, nt_b: int, seed: int, ks: int = 3, vs: int = 3, rescale_p: float = 0.3,
-        max_steps: int = 400000) -> None:
+        max_steps: int = 400000, convert: bool = False) -> None:
     rng = random.Random(seed)
     nts = [nt_a, nt_b]
     ntiles = nts[1] if nts[1] > 0 else nts[0]
@@ -62,6 +66,7 @@ def run(nt_a: int, nt_b: int, seed: int, ks: int = 3, vs: int = 3, rescale_p: fl
     for i in range(vs):
         bar(f"v_full{i}")
         bar(f"v_free{i}", 2)
+        bar(f"v_conv{i}")
     bar("tail")
     for w in range(2):
         for b in range(2):
@@ -79,6 +84,7 @@ def run(nt_a: int, nt_b: int, seed: int, ks: int = 3, vs: int = 3, rescale_p: fl
     s_ready, s_read, p_ready, pv_done = set(), set(), set(), set()
     k_stage, v_stage, k_landed, v_landed = {}, {}, set(), set()
     tail_zeroed = set()
+    converted = set()
     zero_tail = rng.random() < 0.5
     owner = 1 if nts[1] > 0 else 0
 
@@ -117,8 +123,11 @@ def run(nt_a: int, nt_b: int, seed: int, ks: int = 3, vs: int = 3, rescale_p: fl
             yield None
 
         def pv(j):
-            yield from wait(f"v_full{j % vs}", j // vs)
-            if zero_tail and j == ntiles - 1:
+            if convert:
+                yield from wait(f"v_conv{j % vs}", j // vs)
+            else:
+                yield from wait(f"v_full{j % vs}", j // vs)
+            if zero_tail and j == ntiles - 1 and not convert:
                 if w == owner:
                     tail_zeroed.add(j)
                     bars["tail"].arrive()
@@ -162,7 +171,19 @@ def run(nt_a: int, nt_b: int, seed: int, ks: int = 3, vs: int = 3, rescale_p: fl
             yield from wait(f"o_done{w}{(nts[w] - 1) & 1}", (nts[w] - 1) >> 1)
             assert all((w, j) in pv_done for j in range(nts[w])), "epilogue before every PV completed"
 
-    roles = [load(), issuer(0), issuer(1), softmax(0), softmax(1)]
+    def converter():
+        for j in range(ntiles):
+            yield from wait(f"v_full{j % vs}", j // vs)
+            assert v_stage[j % vs] == j and j in v_landed, f"V({j}) converted before it landed"
+            for _ in range(rng.randint(1, 30)):
+                yield None
+            if zero_tail and j == ntiles - 1:
+                tail_zeroed.add(j)
+            converted.add(j)
+            bars[f"v_conv{j % vs}"].arrive()
+            yield None
+
+    roles = [load(), issuer(0), issuer(1), softmax(0), softmax(1)] + ([converter()] if convert else [])
     alive = [True] * len(roles)
     steps = 0
     while any(alive):
@@ -200,6 +221,7 @@ def run(nt_a: int, nt_b: int, seed: int, ks: int = 3, vs: int = 3, rescale_p: fl
                     assert v_stage[j % vs] == j and j in v_landed, f"PV({w},{j}) without its V tile"
                     assert (w, j) in p_ready, f"PV({w},{j}) before P was written"
                     assert not (zero_tail and j == ntiles - 1) or j in tail_zeroed
+                    assert not convert or j in converted, f"PV({w},{j}) before V({j}) was converted"
         order = list(range(len(roles)))
         rng.shuffle(order)
         for i in order:

@@ -174,6 +174,26 @@ def test_prefill_bad_context_len_and_block_id(pa):
     assert (code, detail) == (1, 10 ** 6)
 
 
+def test_prefill_v_out_of_range_reported(pa, orc):
+    # bf16 caches: V enters P V as fp16 times 2^-8, which holds every |v| < 2^24.
+    # One attended V element of sequence 1 at 2^25 is reported (detail = the
+    # sequence); sequence 0's rows stay within tolerance of the oracle.
+    cfg = inputs.DecodeConfig("prefill_range", 73, 2, 8, 2, 128, "bf16")
+    case = inputs.make_prefill_case(cfg, chunk_lens=[20, 20], prefix_lens=[5, 30])
+    vc = case.v_cache.clone()
+    blk = int(case.block_tables[1, 0])
+    vc[blk, 3, 1, 7] = 2.0 ** 25
+    ref = orc.paged_prefill(case.q, case.k_cache, vc, case.block_tables, case.context_lens, case.query_start_loc,
+                            case.scale)
+    pa.get_device_error(clear=True)
+    out = pa.prefill(case.q.cuda(), case.k_cache.cuda(), vc.cuda(), case.block_tables.cuda(),
+                     case.context_lens.cuda(), case.query_start_loc.cuda(), case.scale, max_query_len=20)
+    code, detail = pa.get_device_error(clear=True)
+    assert (code, detail) == (6, 1)
+    rows0 = slice(0, int(case.query_start_loc[1]))
+    _close(out[rows0], ref[rows0], "sequence 0")
+
+
 def test_prefill_empty_chunks(pa, orc):
     # sequences with no query rows in this step are skipped; others unaffected
     cfg = inputs.DecodeConfig("prefill_empty", 81, 4, 8, 2, 128, "f16")

@@ -8,8 +8,8 @@ for S = Q K^T (both operands K-major) and O += P V (V MN-major).  The 128-byte
 swizzle exchanges the 16-byte chunks of each 128-byte row by the row's index
 within its 1024-byte atom.  Tile elements here are unique 16-bit identifiers,
 so every operand the descriptors describe must read back exactly the matrix
-the product needs.  Also checked: where P's two 16-bit parts land in tensor
-memory for the products that read them, and the accuracy of the hi + lo split.
+the product needs.  Also checked: where P's fp16 pairs land in tensor
+memory for the products that read them, and the accuracy of P and V in fp16.
 """
 import numpy as np
 
@@ -90,38 +90,44 @@ def test_kv_tiles_and_product_descriptors():
 
 
 def test_p_columns_in_tensor_memory():
-    """The softmax stores P(j) over S(j): hi pairs (tokens 2k, 2k+1) at column k,
-    lo pairs at column 32 + k, the lower token in the low half.  The product for
-    tokens 16kk..16kk+15 of part p reads columns p*32 + 8kk .. + 7."""
+    """The softmax stores P(j) over S(j) as fp16 pairs (tokens 2k, 2k+1) at
+    column k, the lower token in the low half.  The product for tokens
+    16kk..16kk+15 reads columns 8kk .. 8kk + 7."""
     col_of = {}
-    for part in range(2):
-        for k in range(32):
-            for h in range(2):
-                col_of[(part, 2 * k + h)] = (part * 32 + k, h)
-    for part in range(2):
-        for kk in range(KV // 16):
-            cols = [part * 32 + kk * 8 + c for c in range(8)]
-            tokens = [(c - part * 32) * 2 + h for c in cols for h in range(2)]
-            assert tokens == list(range(16 * kk, 16 * kk + 16))
-            assert all(col_of[(part, t)][0] in cols for t in tokens)
+    for k in range(32):
+        for h in range(2):
+            col_of[2 * k + h] = (k, h)
+    for kk in range(KV // 16):
+        cols = [kk * 8 + c for c in range(8)]
+        tokens = [c * 2 + h for c in cols for h in range(2)]
+        assert tokens == list(range(16 * kk, 16 * kk + 16))
+        assert all(col_of[t][0] in cols for t in tokens)
 
 
-def test_hi_lo_split_accuracy():
-    """hi = p truncated to bf16, lo = the exact remainder truncated to bf16:
-    |p - hi - lo| < 2^-15 |p| over p in (0, 2^8] (the lazy-rescale range)."""
+def test_fp16_p_and_v_conversion():
+    """P in fp16 (nearest): relative rounding <= 2^-11 over the lazy-rescale
+    range (0, 2^8], and absolute <= 2^-25 where it is subnormal.  bf16 V
+    times 2^-8 in fp16: exact for every bf16 value with 2^-6 <= |v| < 2^24,
+    within 2^-17 absolute below that, and out of range (inf) from 2^24 up."""
     rng = np.random.default_rng(5)
     p = np.concatenate([rng.uniform(0, 1, 200000), rng.uniform(1, 256, 50000),
                         2.0 ** rng.uniform(-40, 0, 50000)]).astype(np.float32)
-    p = p[p > 0]
-    trunc = lambda x: (x.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
-    hi = trunc(p)
-    rem = (p - hi).astype(np.float32)              # exact: hi holds p's top bits
-    assert np.array_equal(rem.astype(np.float64), p.astype(np.float64) - hi.astype(np.float64))
-    lo = trunc(rem)
-    err = np.abs(p.astype(np.float64) - hi.astype(np.float64) - lo.astype(np.float64))
-    assert (err < 2.0 ** -15 * p.astype(np.float64)).all()
-    # one 16-bit part alone would not do: its error reaches 2^-8 relative
-    assert (np.abs(p.astype(np.float64) - hi.astype(np.float64)) / p).max() > 2.0 ** -9
+    h = p.astype(np.float16).astype(np.float64)
+    err = np.abs(h - p.astype(np.float64))
+    assert (err <= np.maximum(2.0 ** -11 * p, 2.0 ** -25)).all()
+    # every bf16 bit pattern: exponent fields 1..254 (finite, normal), both signs
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    v = (bits << 16).view(np.float32)
+    v = v[np.isfinite(v)]
+    with np.errstate(over="ignore"):
+        scaled = (v * np.float32(2.0 ** -8)).astype(np.float16)
+    back = scaled.astype(np.float64) * 256.0
+    a = np.abs(v.astype(np.float64))
+    exact = (a >= 2.0 ** -6) & (a < 2.0 ** 24)
+    assert np.array_equal(back[exact], v.astype(np.float64)[exact])
+    small = a < 2.0 ** -6
+    assert (np.abs(back[small] - v.astype(np.float64)[small]) <= 2.0 ** -17).all()
+    assert np.isinf(back[a >= 2.0 ** 24 + 2.0 ** 17]).all()
 
 
 def test_emulation_catches_a_wrong_stride():

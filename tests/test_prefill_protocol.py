@@ -2,7 +2,8 @@
 model (tests/prefill_protocol_model.py): every run ends, no mbarrier wait sees
 a phase early, and every tensor-core product finds its operands in place --
 for query-tile pairs whose KV walks have equal and different lengths, and for
-one query tile only."""
+one query tile only; with and without the converter role that rewrites bf16
+V tiles as fp16 before the PV products read them."""
 import pytest
 
 from prefill_protocol_model import run
@@ -10,10 +11,11 @@ from prefill_protocol_model import run
 SHAPES = [(1, 1), (1, 2), (2, 2), (3, 4), (7, 8), (12, 12), (5, 0), (2, 0), (20, 21)]
 
 
+@pytest.mark.parametrize("convert", [False, True])
 @pytest.mark.parametrize("nt_a,nt_b", SHAPES)
-def test_protocol_runs_clean(nt_a, nt_b):
+def test_protocol_runs_clean(nt_a, nt_b, convert):
     for seed in range(12):
-        run(nt_a, nt_b, seed)
+        run(nt_a, nt_b, seed, convert=convert)
 
 
 PLANTED = {
@@ -24,6 +26,9 @@ PLANTED = {
     # QK(j) waits for PV(j-1) on the other parity's barrier
     "wrong_pv_phase": ('yield from wait(f"o_done{w}{j & 1}", (j - 2) >> 1)',
                        'yield from wait(f"o_done{w}{(j - 1) & 1}", (j - 1) >> 1)'),
+    # bf16 caches: PV waits for the landed V tile instead of the converted one
+    "pv_before_conversion": ('                yield from wait(f"v_conv{j % vs}", j // vs)\n',
+                             '                yield from wait(f"v_full{j % vs}", j // vs)\n'),
 }
 
 
@@ -40,7 +45,7 @@ def test_model_catches_planted_mistakes(mistake):
     caught = 0
     for seed in range(20):
         try:
-            ns["run"](6, 7, seed, max_steps=60000)
+            ns["run"](6, 7, seed, max_steps=60000, convert=mistake == "pv_before_conversion")
         except AssertionError:
             caught += 1
     assert caught > 0
