@@ -795,12 +795,12 @@ def run_reference_prefill(args, world, rank):
 
 
 class PackedInputs:
-    """All of a step's input tensors in ONE pinned host buffer, and two device
-    buffers of the same layout (each tensor at a 256-byte-aligned offset), so a
-    step's inputs move with one host->device copy; views into a device buffer
-    feed the calls."""
+    """All of a step's input tensors in ONE pinned host buffer, and `sets`
+    device buffers of the same layout (each tensor at a 256-byte-aligned
+    offset), so a step's inputs move with one host->device copy; views into a
+    device buffer feed the calls."""
 
-    def __init__(self, tensors, device):
+    def __init__(self, tensors, device, sets=2):
         self.offsets, off = {}, 0
         for n, t in tensors.items():
             self.offsets[n] = off
@@ -810,7 +810,7 @@ class PackedInputs:
         for n, t in tensors.items():
             o, nb = self.offsets[n], t.numel() * t.element_size()
             self.host[o:o + nb].copy_(t.contiguous().reshape(-1).view(torch.uint8))
-        self.dev = [torch.empty(off, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.dev = [torch.empty(off, dtype=torch.uint8, device=device) for _ in range(sets)]
         self.views = []
         for buf in self.dev:
             v = {}
@@ -825,25 +825,27 @@ def pipelined_e2e(step, host, out_like, steps, warmup):
     (name -> host tensor, packed into one pinned buffer) to the device in one
     copy, makes the step's C calls (arguments marshalled once, the call made
     directly, no per-call Python checks) and copies the output back into pinned
-    host memory.  Two sets of device inputs and outputs alternate between steps,
-    with one copy stream per direction, so that step k's copies overlap the
-    kernels of step k-1 (as a serving loop would run them); every copy of every
-    timed step lies inside the timed region.  Also reports the host time of
-    issuing a step (a short burst timed with the GPU idle at its start)."""
+    host memory.  Three sets of device inputs and outputs rotate between steps,
+    with one copy stream per direction, so that step k's input copy may run
+    during the kernels of steps k-2 and k-1 and its output copy during those of
+    step k+1 (as a serving loop would run them); every copy of every timed step
+    lies inside the timed region.  Also reports the host time of issuing a step
+    (a short burst timed with the GPU idle at its start)."""
+    NSETS = 3
     compute = torch.cuda.current_stream()
     device = out_like.device
     h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
-    packed = PackedInputs(host, device)
-    outs = [torch.empty_like(out_like) for _ in range(2)]
-    out_host = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory() for _ in range(2)]
-    calls = [step.raw_calls(packed.views[i], outs[i], compute) for i in range(2)]
-    loaded = [torch.cuda.Event() for _ in range(2)]     # inputs of set i on the device
-    consumed = [torch.cuda.Event() for _ in range(2)]   # kernels that read set i (and write its output) done
-    drained = [torch.cuda.Event() for _ in range(2)]    # output of set i copied to the host
+    packed = PackedInputs(host, device, NSETS)
+    outs = [torch.empty_like(out_like) for _ in range(NSETS)]
+    out_host = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory() for _ in range(NSETS)]
+    calls = [step.raw_calls(packed.views[i], outs[i], compute) for i in range(NSETS)]
+    loaded = [torch.cuda.Event() for _ in range(NSETS)]     # inputs of set i on the device
+    consumed = [torch.cuda.Event() for _ in range(NSETS)]   # kernels that read set i (and write its output) done
+    drained = [torch.cuda.Event() for _ in range(NSETS)]    # output of set i copied to the host
 
     def one(k):
-        i = k & 1
-        h2d_s.wait_event(consumed[i])                   # the step two back is done with these inputs
+        i = k % NSETS
+        h2d_s.wait_event(consumed[i])                   # the step NSETS back is done with these inputs
         with torch.cuda.stream(h2d_s):
             packed.dev[i].copy_(packed.host, non_blocking=True)
         loaded[i].record(h2d_s)
@@ -860,7 +862,7 @@ def pipelined_e2e(step, host, out_like, steps, warmup):
         drained[i].record(d2h_s)
 
     def loop(n):
-        for i in range(2):
+        for i in range(NSETS):
             consumed[i].record(compute)
             drained[i].record(compute)
         h2d_s.wait_stream(compute)
@@ -870,7 +872,7 @@ def pipelined_e2e(step, host, out_like, steps, warmup):
         compute.wait_stream(h2d_s)
         compute.wait_stream(d2h_s)
 
-    loop(max(2, warmup))
+    loop(max(NSETS, warmup))
     torch.cuda.synchronize()
     burst = min(steps, 32)
     t0 = time.perf_counter()
@@ -884,9 +886,9 @@ def pipelined_e2e(step, host, out_like, steps, warmup):
     torch.cuda.synchronize()
     d2h = out_host[0].numel() * out_host[0].element_size()
     return {"ms": a.elapsed_time(b), "h2d": packed.nbytes, "d2h": d2h, "host_us": round(host_us, 2),
-            "last_out_host": out_host[(steps - 1) & 1],
+            "last_out_host": out_host[(steps - 1) % NSETS],
             "path": "one packed pinned->device copy, direct C-ABI calls, one device->pinned copy per step; "
-                    "two buffer sets alternate so copies overlap the previous step's kernels"}
+                    "three buffer sets rotate so copies overlap the neighbouring steps' kernels"}
 
 
 def run_e2e(case, step, steps, warmup, device):
