@@ -241,7 +241,7 @@ pa_status_t pa_decode_append(void *out, const void *q, const void *key, const vo
  * Computed on the tensor cores (tcgen05) with fp32 accumulation; the softmax
  * weights enter P V as fp16 (relative rounding <= 2^-11), and so does V: bf16
  * caches are converted in shared memory, scaled by 2^-8 (exact for every bf16
- * |v| < 2^24; smaller magnitudes keep an absolute accuracy of 2^-17), the
+ * value with 2^-6 <= |v| < 2^24, within 2^-17 absolute below 2^-6), the
  * scale undone in the output.  Device-side errors: PA_DEV_BAD_CONTEXT_LEN (n_b
  * < 0, n_b > max_query_len, L_b < n_b or L_b > max_blocks_per_seq * 16:
  * sequence skipped), PA_DEV_BAD_BLOCK_ID (the block reads as zeros),

@@ -24,7 +24,11 @@
 //                   tiles, online max/sum in base 2 (O rescaled in tensor
 //                   memory only when a row's max grows by more than 2^8), P
 //                   written back over its scores in tensor memory as fp16
-//                   (relative rounding <= 2^-11);
+//                   (relative rounding <= 2^-11); after the last tile, O / l
+//                   staged through the tile's Q buffer (free once its last QK
+//                   has completed) and copied out with coalesced 16-byte
+//                   stores (a warp store covers two whole output rows instead
+//                   of one 16-byte piece of 32 rows);
 //   warps 8, 10     tensor-core issue, one thread per query tile: S = Q K^T
 //                   (M=128 N=64, 8 x K=16, both operands in shared memory)
 //                   into a double-buffered S, and O += P V (M=128 N=128,
@@ -39,9 +43,12 @@
 //                   the rows, 128-byte swizzled) into rings of 3 stages each,
 //                   block ids read from the block table one per lane;
 //   warps 12-15     bf16 caches: rewrite each landed V tile in place as fp16
-//                   times 2^-8 (exact for |v| < 2^24) and zero the rows past
-//                   the context end, then hand it to the issuers; f16 caches:
-//                   idle (as are warp 11 and lanes 1-31 of warps 8 and 10).
+//                   times 2^-8 (exact for 2^-6 <= |v| < 2^24, within 2^-17
+//                   below) and zero the rows past the context end, then hand
+//                   it to the issuers; f16 caches: idle (as are warp 11 and
+//                   lanes 1-31 of warps 8 and 10).
+// Before the barrier set-up the softmax warps already load their Q rows and the
+// TMA warp its first 32 block ids, so that those loads overlap the set-up.
 // Roles hand over through mbarriers (one arrival per warp) only; every wait is
 // bounded, and a role that gives up raises a CTA-wide abort so that the others
 // stop waiting.  Each barrier is waited on by parity, so no barrier may complete
@@ -157,6 +164,18 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// AND of `pred` over the 128 threads of one softmax warpgroup (named barrier kId).
+template <int kId>
+__device__ __forceinline__ bool warpgroup_all(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred p, %2, 128, p;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "n"(kId)
+      : "memory");
+  return r != 0;
+}
+
 template <typename T, int G>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     pa_prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -190,6 +209,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const long long cta = blockIdx.x + static_cast<long long>(gridDim.x) * (blockIdx.y + static_cast<long long>(gridDim.y) * blockIdx.z);
   const unsigned long long wait_limit = wait_limit_for(p.stall_cta, cta);
   const bool stall_here = p.stall_cta != 0 && cta == p.stall_cta - 1;
+  if (warp == kPrefillLoadWarp && lane == 0) {   // kernel parameters: independent of the previous grid
+    prefetch_tensor_map(&tm_k);
+    prefetch_tensor_map(&tm_v);
+  }
   pdl_wait();
   pdl_trigger();
 
@@ -220,9 +243,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int nblk = pos_last_all / kBlockSize + 1;          // cache blocks covering tokens 0 .. pos_last_all
   const int32_t *bt_row = p.block_tables + static_cast<size_t>(b) * p.max_blocks_per_seq;
 
+  // ---- started before the barrier set-up: the Q rows' loads (softmax
+  // warps) and the first 32 block ids (TMA warp)
+  uint4 qx[16];
+  int tma_grp = -1, tma_id = 0;
+  if (warp < kPrefillMmaWarp) {
+    const int w = warp >> 2;
+    const int q0 = (ct * NT + w) * QT;
+    const int nq = max(0, min(QT, n - q0));
+    const T *qg = reinterpret_cast<const T *>(p.q);
+    const int c = tid & 15;              // this thread's 16-byte chunk of every row it moves
+    const int row0 = (tid & 127) >> 4;   // rows row0, row0 + 8, ...
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {   // every load in flight before the first store
+      const int row = row0 + 8 * k;
+      const int i = row / G, hl = row % G;
+      qx[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < nq)
+        qx[k] = *reinterpret_cast<const uint4 *>(
+            qg + (static_cast<size_t>(qs + q0 + i) * p.num_heads + g * G + hl) * D + c * 8);
+    }
+  } else if (warp == kPrefillLoadWarp) {
+    tma_grp = 0;
+    tma_id = static_cast<int>(p.num_blocks);   // past the end of the pool: the box reads zeros
+    if (lane < nblk) {
+      const int v = bt_row[lane];
+      if (v < 0 || v >= p.num_blocks) record_error(1 /*PA_DEV_BAD_BLOCK_ID*/, v);
+      else tma_id = v;
+    }
+  }
   if (tid == 0) {
-    prefetch_tensor_map(&tm_k);
-    prefetch_tensor_map(&tm_v);
     for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_free[i], NT);   // one arrival per issuing thread
@@ -256,32 +306,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // ---- Q tiles -> shared memory, K-major 128-byte swizzled: [d half][row][128 B].
-  // The TMA warp streams K/V meanwhile; only the issuing warps wait for Q
-  // (named barrier 1: the softmax warpgroups and warps 8 and 10).
+  // ---- Q tiles -> shared memory (rows loaded above), K-major 128-byte swizzled:
+  // [d half][row][128 B].  The TMA warp streams K/V meanwhile; only the issuing
+  // warps wait for Q (named barrier 1: the softmax warpgroups and warps 8 and 10).
   if (warp < kPrefillMmaWarp) {
     const int w = warp >> 2;
-    const int q0 = (ct * NT + w) * QT;
-    const int nq = max(0, min(QT, n - q0));
-    const T *qg = reinterpret_cast<const T *>(p.q);
     uint8_t *q_s = smem + SM::kQ + w * SM::kQTileBytes;
-    const int c = tid & 15;              // this thread's 16-byte chunk of every row it moves
-    const int row0 = (tid & 127) >> 4;   // rows row0, row0 + 8, ...
-    uint4 x[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {   // every load in flight before the first store
-      const int row = row0 + 8 * k;
-      const int i = row / G, hl = row % G;
-      x[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (i < nq)
-        x[k] = *reinterpret_cast<const uint4 *>(
-            qg + (static_cast<size_t>(qs + q0 + i) * p.num_heads + g * G + hl) * D + c * 8);
-    }
+    const int c = tid & 15;
+    const int row0 = (tid & 127) >> 4;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       const int row = row0 + 8 * k;
       *reinterpret_cast<uint4 *>(q_s + (c >> 3) * (kPrefillRows * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
-          x[k];
+          qx[k];
     }
     fence_proxy_async_smem();   // the generic stores of Q are read by the tensor cores
   }
@@ -296,7 +333,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   if (warp == kPrefillLoadWarp) {
     // ================================================================ TMA producer
-    int grp = -1, my_id = 0;
+    int grp = tma_grp, my_id = tma_id;
     auto issue = [&](int j, bool is_v) {   // all lanes; j uniform
       const int want = (4 * j) >> 5;
       if (want != grp) {
@@ -442,8 +479,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if constexpr (PK::kConvertV) {
       // ================================================================ V converter (bf16 caches)
       // Every landed V tile is rewritten in place as fp16 times 2^-8 (exact for
-      // |v| < 2^24, the kernel's stated range; larger magnitudes are recorded as
-      // PA_DEV_VALUE_RANGE), and the rows of tokens at or past the context end
+      // 2^-6 <= |v| < 2^24, within 2^-17 absolute below; |v| >= 2^24 is out of
+      // the kernel's stated range and recorded as PA_DEV_VALUE_RANGE), and the rows of tokens at or past the context end
       // (stale slots of the last block, possibly NaN) become zero, so that
       // 0 * V stays 0.  The element positions do not move, so the tile keeps
       // its swizzled layout.  Four warps, 8 16-byte chunks a lane per tile;
@@ -574,25 +611,39 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tb[2 + (j & 1)]);   // P(j) written (and O rescaled)
     }
-    if (ok && ntw > 0) {
-      // -- epilogue: O / l -> out
+    if (ntw > 0) {
+      // -- epilogue: O / l -> out, staged through this tile's Q buffer (its
+      // last QK has completed: the softmax saw its scores).  Each thread puts
+      // its row in shared memory (16-byte chunk c of row r at position
+      // c ^ (r & 15): four wavefronts a warp store), then the warpgroup copies
+      // the valid rows out with consecutive lanes on consecutive chunks, so
+      // that a warp store covers two whole 256-byte rows.
       wait(&tb[4 + ((ntw - 1) & 1)], ((ntw - 1) >> 1) & 1);   // the last PV (and so every PV) done
+      uint8_t *stage = smem + SM::kQ + w * SM::kQTileBytes;
       if (ok) {
         const float inv = (PK::kConvertV ? 256.f : 1.f) / l_run;   // V entered P V scaled by 2^-8
-        T *orow = reinterpret_cast<T *>(p.out) +
-                  (static_cast<size_t>(qs + q0 + i_row) * p.num_heads + g * G + r % G) * D;
-        const bool row_valid = i_row < nq;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           float o[32];
           tmem_ld32(t_o + c, o);
-          if (row_valid) {
 #pragma unroll
-            for (int k = 0; k < 32; k += 8)
-              *reinterpret_cast<uint4 *>(orow + c + k) =
-                  make_uint4(PK::pack(o[k] * inv, o[k + 1] * inv), PK::pack(o[k + 2] * inv, o[k + 3] * inv),
-                             PK::pack(o[k + 4] * inv, o[k + 5] * inv), PK::pack(o[k + 6] * inv, o[k + 7] * inv));
-          }
+          for (int k = 0; k < 32; k += 8)
+            *reinterpret_cast<uint4 *>(stage + r * 256 + ((((c + k) >> 3) ^ (r & 15)) << 4)) =
+                make_uint4(PK::pack(o[k] * inv, o[k + 1] * inv), PK::pack(o[k + 2] * inv, o[k + 3] * inv),
+                           PK::pack(o[k + 4] * inv, o[k + 5] * inv), PK::pack(o[k + 6] * inv, o[k + 7] * inv));
+        }
+      }
+      // every warp of the warpgroup takes the barrier, and copies out only if all staged their rows
+      const bool all_ok = w == 0 ? warpgroup_all<2>(ok) : warpgroup_all<3>(ok);   // named barriers 2, 3
+      if (all_ok) {
+        T *out_t = reinterpret_cast<T *>(p.out);
+        const int units = nq * G * 16;   // 16-byte chunks of the valid rows
+#pragma unroll 4
+        for (int u = r; u < units; u += 128) {
+          const int rr = u >> 4, ch = u & 15;
+          const uint4 v = *reinterpret_cast<const uint4 *>(stage + rr * 256 + ((ch ^ (rr & 15)) << 4));
+          *reinterpret_cast<uint4 *>(out_t + (static_cast<size_t>(qs + q0 + rr / G) * p.num_heads + g * G + rr % G) * D +
+                                     ch * 8) = v;
         }
       }
     }

@@ -135,3 +135,58 @@ def test_emulation_catches_a_wrong_stride():
     blocks_v = [ids(16, 128, 7000 + 1000 * i) for i in range(4)]
     V, smv = np.vstack(blocks_v), _tma_tile(blocks_v)
     assert not np.array_equal(read_mnmajor(smv, 0, 16, 1024, 128), V[0:16, :])
+
+
+def _bank_degree(byte_addrs):
+    """Wavefronts of one warp's 16-byte shared-memory accesses: the largest
+    number of distinct 4-byte words any of the 32 banks must serve."""
+    words = {(a // 4 + i) for a in byte_addrs for i in range(4)}
+    per_bank = {}
+    for wd in words:
+        per_bank[wd % 32] = per_bank.get(wd % 32, 0) + 1
+    return max(per_bank.values())
+
+
+def stage_addr(r, ch):
+    """Epilogue staging in the Q buffer: 16-byte chunk ch of output row r."""
+    return r * 256 + ((ch ^ (r & 15)) << 4)
+
+
+def test_epilogue_staging_and_copy_out():
+    """O / l goes through the tile's 32 KiB Q buffer: thread r (the row) writes
+    its 16 chunks at stage_addr(r, ch); the warpgroup then copies unit u (row
+    u >> 4, chunk u & 15) from there to the output row of query r // G, head
+    g*G + r % G.  Checked: the staging is a permutation of the buffer, every
+    warp access takes the minimum 4 wavefronts, the copy reads back exactly
+    what each row wrote, and a warp store covers at most 4 128-byte lines
+    (the row-per-thread store it replaces covers 32)."""
+    addrs = sorted(stage_addr(r, ch) for r in range(128) for ch in range(16))
+    assert addrs == list(range(0, 32768, 16))
+    for q in range(4):                      # warp q of the warpgroup writes rows 32q .. 32q + 31
+        for ch in range(16):
+            assert _bank_degree([stage_addr(32 * q + l, ch) for l in range(32)]) == 4
+    for G in (1, 2, 4, 8):
+        Hq, g, qs, q0 = 32, 1, 5, 0
+        QT = 128 // G
+        for nq in (QT, 1, QT - 1 if QT > 1 else 1):
+            stage = {}
+            for r in range(128):
+                for ch in range(16):
+                    stage[stage_addr(r, ch)] = (r, ch)
+            units = nq * G * 16
+            seen = set()
+            for base in range(0, units, 32):    # one warp instruction: 32 consecutive units
+                lanes = range(base, min(base + 32, units))
+                assert _bank_degree([stage_addr(u >> 4, u & 15) for u in lanes]) <= 4
+                lines = set()
+                for u in lanes:
+                    rr, ch = u >> 4, u & 15
+                    assert stage[stage_addr(rr, ch)] == (rr, ch)
+                    elem = ((qs + q0 + rr // G) * Hq + g * G + rr % G) * 128 + ch * 8
+                    seen.add((rr, ch))
+                    lines.add(elem * 2 // 128)
+                assert len(lines) <= 4
+            assert seen == {(r, ch) for r in range(nq * G) for ch in range(16)}
+    # the store it replaces: each lane its own row, one 16-byte chunk per instruction
+    old = {(((r // 4) * 32 + 4 + r % 4) * 128 * 2) // 128 for r in range(32)}
+    assert len(old) == 32
