@@ -36,9 +36,12 @@
 //                   memory), QK(j+1) before PV(j); the tensor pipe runs one
 //                   query tile's products while the other's issuer waits.  A
 //                   product costs about the same below N=256 whatever its
-//                   width, so the kernel is bound by its count of products:
+//                   width (56-64 cycles at N=64 and at N=128, 128 at N=256);
 //                   one fp16 pass of P V instead of two bf16 ones (hi + lo)
-//                   takes a quarter of them away;
+//                   takes a quarter of them away.  The pipe is busy about
+//                   half of each step: the step is set by each query tile's
+//                   chain through its two S buffers, QK(j+2) after PV(j)
+//                   after softmax(j), and by the hand-overs;
 //   warp 9          TMA: K and V tiles (four 2 KiB boxes per 128-byte half of
 //                   the rows, 128-byte swizzled) into rings of 3 stages each,
 //                   block ids read from the block table one per lane;
