@@ -12,7 +12,8 @@ Roles, as in the kernel:
   whose query tile does not reach a KV tile still arrives once on its stages;
 * one softmax role per query tile waits for S_w(j), sometimes rescales O (then
   waits for PV_w(j-1)), and hands P_w(j) over; the epilogue waits for the
-  last PV;
+  last PV, then stages O in the tile's Q buffer, which every QK_w product
+  must have finished reading;
 * with `convert` (bf16 caches) a converter role takes every landed V tile,
   rewrites it in place as fp16 (and zeroes the rows past the context end of
   the last tile), and hands it to the issuers on its own barrier per stage;
@@ -170,6 +171,7 @@ def run(nt_a: int, nt_b: int, seed: int, ks: int = 3, vs: int = 3, rescale_p: fl
         if nts[w] > 0:
             yield from wait(f"o_done{w}{(nts[w] - 1) & 1}", (nts[w] - 1) >> 1)
             assert all((w, j) in pv_done for j in range(nts[w])), "epilogue before every PV completed"
+            assert all((w, j) in s_ready for j in range(nts[w])), "Q buffer reused before every QK completed"
 
     def converter():
         for j in range(ntiles):
